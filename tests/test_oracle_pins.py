@@ -1,0 +1,379 @@
+"""Pins of the fp64 oracle against what the pages and the mathematics fix.
+
+None of these checks re-types the oracle's own formula: each uses a closed form,
+exact rational arithmetic, brute force on tiny inputs, a second formulation or a
+library routine on a special case, so that a dropped term, a wrong sign or
+index, or a transposed operand in the oracle fails at least one of them.
+"""
+
+import itertools
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import stem_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _rand(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- encodings
+
+def test_bf16_decode_matches_library_and_known_values():
+    bits = np.arange(0, 1 << 16, 7, dtype=np.uint32).astype(np.uint16)
+    ours = O.bf16_bits_to_f64(bits)
+    lib = torch.from_numpy(bits.astype(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    same = (ours == lib) | (np.isnan(ours) & np.isnan(lib))
+    assert same.all()
+    assert O.bf16_bits_to_f64(np.array([0x3F80, 0xC000, 0x0000, 0x4049], dtype=np.uint16)).tolist() == \
+        [1.0, -2.0, 0.0, 3.140625]
+
+
+def test_e4m3_decode_matches_library_and_format_extremes():
+    b = np.arange(256, dtype=np.uint8)
+    ours = O.e4m3_bytes_to_f64(b)
+    lib = torch.from_numpy(b).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    same = (ours == lib) | (np.isnan(ours) & np.isnan(lib))
+    assert same.all()
+    # largest normal 448 = 1.75 * 2^8, smallest subnormal 2^-9, NaN at 0x7F/0xFF
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9
+    assert np.isnan(ours[0x7F]) and np.isnan(ours[0xFF])
+
+
+def test_fp8_dequant_applies_per_head_scale():
+    x = np.array([[[0x38, 0x40], [0x38, 0x40]]], dtype=np.uint8)  # 1.0, 2.0 per head
+    out = O.dequant(x, "fp8", np.array([0.5, 3.0], dtype=np.float32))
+    assert out.tolist() == [[[0.5, 1.0], [3.0, 6.0]]]
+
+
+# ---------------------------------------------------------------- defaults
+
+def test_defaults_match_documented_table():
+    g = json.load(open(os.path.join(GOLDEN, "angelslim_defaults.json")))
+    p = O.Params()
+    assert p.block_size == g["block_size"] and p.stride == g["stride"]
+    assert p.chunk_size == g["chunk_size"] and p.norm == g["norm"]
+    assert p.sink_blocks == g["initial_blocks"] and p.window_blocks == g["window_size"]
+    assert p.mu == g["mu_best"] and p.beta == g["beta_best"]
+
+
+# ---------------------------------------------------------------- TPD budget
+
+def _exact_k(i, nb, rho, mu, relative=True):
+    """k(i) = floor(k_start - k_start (1-mu)/N * i) in exact rationals, with rho
+    and mu taken as the decimals the caller wrote.  Also returns whether the
+    real value sits exactly on an integer (where fp64 rounding may land on
+    either side)."""
+    rho, mu = Fraction(str(rho)), Fraction(str(mu))
+    c = i + 1
+    ks = math.ceil(rho * c) if relative else math.ceil(rho * nb)
+    val = ks - ks * (1 - mu) / nb * i
+    return ks, math.floor(val), val.denominator == 1
+
+
+@pytest.mark.parametrize("rho,mu,nb", [(0.25, 0.7, 256), (0.5, 0.7, 16), (0.25, 0.7, 1024),
+                                       (0.2, 1.0, 512), (0.1, 1.0, 512), (0.25, 0.7, 64),
+                                       (0.3, 0.45, 100), (1.0, 0.7, 37)])
+@pytest.mark.parametrize("relative", [True, False])
+def test_tpd_closed_form_against_exact_rationals(rho, mu, nb, relative):
+    p = O.Params(keep_ratio=rho, mu=mu, budget_mode=O.RELATIVE if relative else O.ABSOLUTE)
+    for i in range(nb):
+        ks, k = O.tpd_k(i, nb, p)
+        eks, ek, on_integer = _exact_k(i, nb, rho, mu, relative)
+        assert ks == eks
+        # fp64 (the fixed evaluation order) may only differ from exact arithmetic
+        # where the exact value is an integer, and then by one step down.
+        if k != ek:
+            assert on_integer and k == ek - 1, (i, k, ek)
+
+
+def test_tpd_endpoints_and_uniform_limit():
+    # i = 0 gives k_start; mu = 1 gives the uniform budget (k_end = mu k_start).
+    for nb in (16, 256, 1000):
+        for rho in (0.1, 0.25, 0.5):
+            p1 = O.Params(keep_ratio=rho, mu=1.0)
+            for i in range(nb):
+                ks, k = O.tpd_k(i, nb, p1)
+                assert k == ks
+            p = O.Params(keep_ratio=rho, mu=0.7)
+            ks0, k0 = O.tpd_k(0, nb, p)
+            assert k0 == ks0 == math.ceil(rho)
+    # absolute mode, i = N: k(N) = floor(mu * k_start) (the page's k_end)
+    p = O.Params(keep_ratio=0.25, mu=0.7, budget_mode=O.ABSOLUTE)
+    nb = 400
+    ks = math.ceil(0.25 * nb)
+    k_end = math.floor(ks - ks * (1 - Fraction("0.7")) / nb * nb)
+    assert k_end == math.floor(Fraction("0.7") * ks)
+
+
+def test_tpd_monotone_in_mu_and_full_density():
+    nb = 300
+    for i in range(nb):
+        ks_prev = -1
+        for mu in (0.1, 0.3, 0.5, 0.7, 0.9, 1.0):
+            _, k = O.tpd_k(i, nb, O.Params(keep_ratio=0.25, mu=mu))
+            assert k >= ks_prev
+            ks_prev = k
+    cu = [0, 128 * 50, 128 * 50 + 300]
+    b = O.budgets(cu, O.Params(keep_ratio=1.0, mu=1.0, sink_blocks=0, window_blocks=1))
+    expect = list(range(1, 51)) + list(range(1, 4))
+    assert b.tolist() == expect
+
+
+def test_forced_blocks_examples():
+    assert O.forced_blocks(0, 4, 4) == [0]
+    assert O.forced_blocks(5, 1, 1) == [0, 5]
+    assert O.forced_blocks(5, 4, 4) == [0, 1, 2, 3, 4, 5]
+    assert O.forced_blocks(9, 1, 2) == [0, 8, 9]
+    assert O.forced_blocks(9, 0, 1) == [9]
+    # budget never below |F| nor above c
+    p = O.Params(keep_ratio=0.05, mu=0.5, sink_blocks=4, window_blocks=4)
+    for i in range(40):
+        b = O.tpd_budget(i, 40, p)
+        assert len(O.forced_blocks(i, 4, 4)) <= b <= i + 1
+
+
+# ---------------------------------------------------------------- selection
+
+def test_selection_equals_subset_brute_force():
+    rng = np.random.default_rng(7)
+    for trial in range(60):
+        i = int(rng.integers(0, 11))
+        c = i + 1
+        S, W = int(rng.integers(0, 3)), int(rng.integers(1, 3))
+        F = O.forced_blocks(i, S, W)
+        b = int(rng.integers(len(F), c + 1))
+        row = rng.permutation(c).astype(np.float64) + rng.random(c) * 0.1  # distinct
+        rest = [j for j in range(c) if j not in F]
+        best, best_set = -math.inf, None
+        for comb in itertools.combinations(rest, b - len(F)):
+            tot = sum(row[j] for j in comb)
+            if tot > best:
+                best, best_set = tot, comb
+        assert O.select_row(row, i, b, S, W) == sorted(F + list(best_set))
+
+
+def test_selection_ties_nan_and_structure():
+    row = np.array([0.0, 5.0, 5.0, 5.0, np.nan, -np.inf, 1.0, 9.0])
+    # i=7, W=1 forces {7}; S=0; budget 3 -> two of {1,2,3} by lowest index
+    assert O.select_row(row, 7, 3, 0, 1) == [1, 2, 7]
+    # NaN ranks like -inf, behind 0.0; tie between NaN(4) and -inf(5) -> index 4
+    assert O.select_row(row, 7, 7, 0, 1) == [0, 1, 2, 3, 4, 6, 7]
+    rng = np.random.default_rng(3)
+    cu = [0, 128 * 24]
+    p = O.Params(keep_ratio=0.3, mu=0.7, sink_blocks=2, window_blocks=3)
+    sc = rng.standard_normal((3, 24, 24))
+    bud, rp, ci = O.select(sc, cu, p)
+    for h in range(3):
+        for i in range(24):
+            r = h * 24 + i
+            sel = ci[rp[r]:rp[r + 1]].tolist()
+            assert len(sel) == bud[r] and sel == sorted(set(sel))
+            assert set(O.forced_blocks(i, 2, 3)) <= set(sel) and max(sel) == i
+    # rho = 1, mu = 1 selects every causal block
+    bud, rp, ci = O.select(sc, cu, O.Params(keep_ratio=1.0, mu=1.0, sink_blocks=0, window_blocks=1))
+    rp2, ci2 = O.full_csr(cu, 3)
+    assert rp.tolist() == rp2.tolist() and ci.tolist() == ci2.tolist()
+
+
+# ---------------------------------------------------------------- scoring
+
+@pytest.mark.parametrize("L,s,d,hq,hkv", [(64, 8, 16, 4, 2), (61, 8, 8, 2, 1), (40, 4, 8, 2, 2)])
+def test_two_scoring_formulations_agree(L, s, d, hq, hkv):
+    q = _rand((L, hq, d), 1)
+    k = _rand((L, hkv, d), 2)
+    A = O.downsampled_scores(q, k, s, 1.5)
+    B = O.downsampled_scores_antidiag(q, k, s, 1.5)
+    assert A.shape == B.shape
+    np.testing.assert_allclose(A, B, rtol=0, atol=1e-12)
+
+
+def test_scoring_closed_form_pairs_anti_diagonal():
+    """q_t = t e0 and k_t = t e0: D[a][b] = sum_u (as+u)(bs+s-1-u)/(sqrt(d) s n),
+    expanded with sum u = s(s-1)/2 and sum u^2 = (s-1)s(2s-1)/6; the main
+    diagonal pairing would give a different value everywhere."""
+    L, s, d, n = 48, 8, 4, 2.0
+    t = np.arange(L, dtype=np.float64)
+    q = np.zeros((L, 1, d)); q[:, 0, 0] = t
+    k = np.zeros((L, 1, d)); k[:, 0, 0] = t
+    D = O.downsampled_scores(q, k, s, n)[0]
+    S1 = s * (s - 1) / 2
+    S2 = (s - 1) * s * (2 * s - 1) / 6
+    for a in range(L // s):
+        for b in range(L // s):
+            A_, B_ = a * s, b * s
+            # (A+u)(B+s-1-u) = A(B+s-1) + u(B+s-1) - A u - u^2
+            tot = s * A_ * (B_ + s - 1) + S1 * (B_ + s - 1) - A_ * S1 - S2
+            assert D[a, b] == pytest.approx(tot / (math.sqrt(d) * s * n), rel=1e-14)
+            diag = s * A_ * B_ + S1 * (A_ + B_) + S2
+            if a == b == 0:
+                continue
+            assert abs(diag - tot) > 0.5
+
+
+def test_block_scores_closed_form_with_bonus():
+    """q_t = e0, k_t = t e0 (so D grows with the key group), and v_t = c_t e0:
+    S_ij = (b_last s + (s-1)/2)/(sqrt(d) n) + beta max(0, ln max c_t^2),
+    b_last the last group of key block j; -inf above the diagonal."""
+    B, s, d = 32, 8, 4
+    L = 4 * B + 20  # partial last block (20 tokens)
+    t = np.arange(L, dtype=np.float64)
+    q = np.zeros((L, 2, d)); q[:, :, 0] = 1.0
+    k = np.zeros((L, 1, d)); k[:, 0, 0] = t
+    c = np.exp(np.sin(t) * 2.0)  # norms spanning both sides of 1
+    v = np.zeros((L, 1, d)); v[:, 0, 0] = c
+    p = O.Params(block_size=B, stride=s, chunk_size=64, beta=0.2, norm=1.0)
+    Sm = O.block_scores(q, k, v, [0, L], p)
+    nb = 5
+    ngv = math.ceil(L / s)
+    for i in range(nb):
+        for j in range(nb):
+            if j > i:
+                assert Sm[0, i, j] == -np.inf
+                continue
+            # key group b contributes sum of its valid token indices; the last
+            # group of the partial block holds tokens 144..151 of which only
+            # 144..147 exist (missing ones count as zero), so it is not the max
+            dval = max(sum(tt for tt in range(b * s, b * s + s) if tt < L)
+                       for b in range(j * (B // s), min((j + 1) * (B // s), ngv))) / (math.sqrt(d) * s)
+            m = max(c[j * B:min((j + 1) * B, L)] ** 2)
+            want = dval + 0.2 * max(0.0, math.log(m))
+            assert Sm[0, i, j] == pytest.approx(want, rel=1e-13)
+            assert Sm[1, i, j] == Sm[0, i, j]
+
+
+def test_value_bonus_special_cases():
+    # ||v||^2 = e^2 -> ln = 2 -> bonus 2 beta; ||v|| < 1 -> bonus 0; zero rows -> 0
+    v = np.zeros((3 * 16, 1, 4))
+    v[:16, 0, 1] = math.e
+    v[16:32, 0, 2] = 0.5
+    b = O.value_bonus(v, [0, 48], 0.2, block=16)
+    assert b[0].tolist() == pytest.approx([0.4, 0.0, 0.0], abs=1e-15)
+
+
+def test_oam_log_form_ranks_like_product_form():
+    """HPC-BSA article §2.2: the log turns the product exp(routing) * magnitude
+    into a sum without changing the ranking.  Top-k by the additive score must
+    equal top-k by exp(max D) * max(1, m_j)^beta on tiny inputs."""
+    rng = np.random.default_rng(11)
+    B, s, d = 16, 4, 8
+    L = 12 * B
+    q = rng.standard_normal((L, 1, d))
+    k = rng.standard_normal((L, 1, d))
+    v = rng.standard_normal((L, 1, d)) * np.exp(rng.standard_normal((L, 1, 1)))
+    p = O.Params(block_size=B, stride=s, chunk_size=64, beta=0.7)
+    Sm = O.block_scores(q, k, v, [0, L], p)[0]
+    D = O.downsampled_scores(q, k, s, 1.0)[0]
+    gpb = B // s
+    for i in range(12):
+        prod = []
+        for j in range(i + 1):
+            mx = D[i * gpb:(i + 1) * gpb, j * gpb:(j + 1) * gpb].max()
+            m = max(np.sum(v[j * B:(j + 1) * B, 0] ** 2, axis=1))
+            prod.append(math.exp(mx) * max(1.0, m) ** 0.7)
+        for kk in range(1, i + 2):
+            top_sum = set(np.argsort(-Sm[i, :i + 1], kind="stable")[:kk].tolist())
+            top_prod = set(np.argsort(-np.array(prod), kind="stable")[:kk].tolist())
+            assert top_sum == top_prod
+
+
+def test_beta_zero_is_pure_routing():
+    rng = np.random.default_rng(5)
+    B, s, d, L = 16, 4, 8, 64
+    q, k = rng.standard_normal((L, 1, d)), rng.standard_normal((L, 1, d))
+    v = rng.standard_normal((L, 1, d)) * 10
+    S0 = O.block_scores(q, k, v, [0, L], O.Params(block_size=B, stride=s, beta=0.0))
+    D = O.downsampled_scores(q, k, s, 1.0)[0]
+    for i in range(4):
+        for j in range(i + 1):
+            assert S0[0, i, j] == D[i * 4:(i + 1) * 4, j * 4:(j + 1) * 4].max()
+
+
+# ---------------------------------------------------------------- attention
+
+def _small_problem(seqlens, hq, hkv, d, seed):
+    rng = np.random.default_rng(seed)
+    T = sum(seqlens)
+    q = rng.standard_normal((T, hq, d))
+    k = rng.standard_normal((T, hkv, d))
+    v = rng.standard_normal((T, hkv, d))
+    cu = np.concatenate([[0], np.cumsum(seqlens)]).tolist()
+    return q, k, v, cu
+
+
+def test_gather_equals_minus_inf_mask():
+    """HPC-BSA article §3.1: skipping a block is the same as -inf scores."""
+    B = 16
+    q, k, v, cu = _small_problem([100, 57], 4, 2, 8, 9)
+    p = O.Params(block_size=B, stride=4, keep_ratio=0.4, mu=0.7, sink_blocks=1, window_blocks=1)
+    S = O.block_scores(q, k, v, cu, p)
+    bud, rp, ci = O.select(S, cu, p)
+    A_o, A_l = O.bsa(q, k, v, cu, rp, ci, p)
+    B_o, B_l = O.bsa_masked(q, k, v, cu, rp, ci, p)
+    np.testing.assert_allclose(A_o, B_o, atol=1e-12)
+    np.testing.assert_allclose(A_l, B_l, atol=1e-12)
+
+
+def test_full_selection_is_dense_causal_attention_sdpa():
+    """rho = 1, mu = 1 keeps every causal block: the result must be ordinary
+    causal softmax attention (torch SDPA in fp64 on CPU, GQA heads repeated)."""
+    B = 16
+    seqlens = [70, 48]
+    q, k, v, cu = _small_problem(seqlens, 4, 2, 8, 4)
+    p = O.Params(block_size=B, stride=4, keep_ratio=1.0, mu=1.0, sink_blocks=0, window_blocks=1,
+                 softmax_scale=0.3)
+    res = O.prefill(q, k, v, cu, p)
+    for s in range(2):
+        o, e = cu[s], cu[s + 1]
+        qt = torch.from_numpy(q[o:e]).permute(1, 0, 2)[None]
+        kt = torch.from_numpy(k[o:e]).permute(1, 0, 2).repeat_interleave(2, 0)[None]
+        vt = torch.from_numpy(v[o:e]).permute(1, 0, 2).repeat_interleave(2, 0)[None]
+        ref = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=True, scale=0.3)
+        np.testing.assert_allclose(res["out"][o:e], ref[0].permute(1, 0, 2).numpy(), atol=1e-12)
+        logits = 0.3 * torch.einsum("htd,hud->htu", qt[0], kt[0])
+        mask = torch.ones(e - o, e - o, dtype=torch.bool).tril()
+        lse = torch.logsumexp(logits.masked_fill(~mask, -math.inf), dim=-1)
+        np.testing.assert_allclose(res["lse"][:, o:e], lse.numpy(), atol=1e-12)
+
+
+def test_first_token_sees_only_itself():
+    B = 16
+    q, k, v, cu = _small_problem([40], 2, 1, 8, 2)
+    p = O.Params(block_size=B, stride=4, keep_ratio=0.5, mu=0.7, sink_blocks=1, window_blocks=1)
+    rp, ci = O.full_csr(cu, 2, B)
+    out, lse = O.bsa(q, k, v, cu, rp, ci, p)
+    sig = 1 / math.sqrt(8)
+    for h in range(2):
+        np.testing.assert_allclose(out[0, h], v[0, 0], atol=1e-15)
+        assert lse[h, 0] == pytest.approx(sig * q[0, h] @ k[0, 0], abs=1e-14)
+
+
+def test_skipped_block_changes_only_its_rows_weights():
+    """Dropping one listed block equals renormalising the softmax without it:
+    O_without = (l_full O_full - l_blk O_blk) / (l_full - l_blk)."""
+    B = 16
+    q, k, v, cu = _small_problem([64], 1, 1, 8, 12)
+    p = O.Params(block_size=B, stride=4)
+    rp_full, ci_full = O.full_csr(cu, 1, B)
+    full_o, full_l = O.bsa(q, k, v, cu, rp_full, ci_full, p)
+    # row of block 3 without key block 1
+    rp = np.array([0, 1, 3, 6, 9])
+    ci = np.array([0, 0, 1, 0, 1, 2, 0, 2, 3])
+    o2, l2 = O.bsa(q, k, v, cu, rp, ci, p)
+    only = np.array([0, 1, 2, 3, 4])
+    rpb = np.array([0, 1, 2, 3, 4])
+    cib = np.array([0, 1, 2, 1])  # block 3's row lists only key block 1
+    ob, lb = O.bsa(q, k, v, cu, rpb, cib, p)
+    t = slice(48, 64)
+    lf, lbk = np.exp(full_l[0, t]), np.exp(lb[0, t])
+    want = (lf[:, None] * full_o[t, 0] - lbk[:, None] * ob[t, 0]) / (lf - lbk)[:, None]
+    np.testing.assert_allclose(o2[t, 0], want, atol=1e-10)
+    np.testing.assert_allclose(np.exp(l2[0, t]), lf - lbk, rtol=1e-12)
