@@ -1,0 +1,491 @@
+#!/usr/bin/env python
+"""Benchmark of the Stem prefill hot path on B200 (one JSON line on rank 0).
+
+Workload (default): one attention layer of a 128K-token prefill shaped like
+Qwen3-8B — 1 x 131072 tokens, 32 query / 8 KV heads, head_dim 128, bf16,
+keep-ratio 0.25, mu 0.7, beta 0.2, 1 sink + 2 window blocks, 128-token blocks,
+scoring stride 8 — on synthetic inputs (N(0,1) queries/keys, the first four
+keys pushed along the mean query, log-normal value norms).
+
+A step is one pass of the whole path: stem_score (value-norm bonus +
+anti-diagonal scoring + block max-pool) -> stem_select (position-decay budget
++ top-k CSR lists) -> stem_bsa_fwd (block-sparse attention), timed with CUDA
+events on the launching stream.  Inputs (Q alone is 1.07 GB) exceed the
+126 MB L2, so no flush is needed between steps.
+
+value = (scoring FLOPs + attention FLOPs of the selected blocks) summed over
+ranks / max-over-ranks step time, in TFLOP/s.  Each rank runs an independent
+layer (weak scaling, no collective on the data path).
+
+`--impl reference` times the fp64 CPU oracle on a bounded sample of the same
+workload instead (there is no other implementation of this method to run).
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "128K prefill attn ms & effective TFLOPS (1×B200, ρ=0.25) vs dense; % of roofline"
+UNIT = "TFLOP/s (scoring + selected-block attention FLOPs per second)"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "bsa_kernel_traffic.txt")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="long128k")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
+    return ap.parse_args(argv)
+
+
+# ---------------------------------------------------------------- distributed plumbing
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def dist_init(backend: str):
+    import torch.distributed as dist
+    rank, world, _ = dist_env()
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world
+
+
+def dist_barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def dist_max(x: float, device="cpu") -> float:
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+    return x
+
+
+def dist_sum(x: float, device="cpu") -> float:
+    import torch
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.SUM)
+        return float(t.item())
+    return x
+
+
+def dist_done():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_id: str):
+        self.device_id = device_id
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        import tempfile
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.device_id, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        smax = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[k] for r in rows for k in range(4) if r[4 + k].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def gpu_device_id(torch) -> str:
+    """nvidia-smi -i argument of the current device: the physical index from
+    CUDA_VISIBLE_DEVICES when it lists indices, else the PCI bus id."""
+    cur = torch.cuda.current_device()
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [x.strip() for x in vis.split(",") if x.strip()]
+    if ids and all(x.isdigit() for x in ids) and cur < len(ids):
+        return ids[cur]
+    props = torch.cuda.get_device_properties(cur)
+    try:
+        return "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+    except AttributeError:
+        return str(cur)
+
+
+def load_peaks():
+    try:
+        pk = json.load(open(PEAKS_FILE))
+        return pk, "measured"
+    except (OSError, ValueError):
+        return FALLBACK_PEAKS, "fallback"
+
+
+def bsa_traffic_per_launch():
+    """dram bytes per launch of the attention kernel from the committed ncu
+    summary, valid only while the kernel source is the one that was profiled."""
+    try:
+        rec = dict(line.split(None, 1) for line in open(TRAFFIC_FILE) if line.strip() and not line.startswith("#"))
+        src = open(os.path.join(ROOT, "block_sparse_attention_stem_b200", "csrc", "k_bsa.cu"), "rb").read()
+        if rec.get("source_sha256", "").strip() != hashlib.sha256(src).hexdigest():
+            return None
+        return float(rec["bytes_per_launch_full_workload"])
+    except (OSError, ValueError, KeyError):
+        return None
+
+
+def describe(w) -> dict:
+    return {
+        "workload": (f"{w.name}: {len(w.seqlens)} x {w.seqlens if len(w.seqlens) > 1 else w.seqlens[0]} tokens, "
+                     f"{w.num_q_heads} Q / {w.num_kv_heads} KV heads, d={w.head_dim}, {w.dtype}, "
+                     f"rho={w.keep_ratio}, mu={w.mu}, beta={w.beta}, sink {w.sink_blocks}, window "
+                     f"{w.window_blocks}, block {w.block_size}, stride {w.stride}"),
+        "seq_len": max(w.seqlens),
+        "total_tokens": w.total_tokens,
+        "num_q_heads": w.num_q_heads,
+        "num_kv_heads": w.num_kv_heads,
+        "l2": "inputs larger than L2 (Q alone %.2f GB > 126 MB); no flush" % (
+            w.total_tokens * w.num_q_heads * w.head_dim * (2 if w.dtype == "bf16" else 1) / 1e9),
+    }
+
+
+# ---------------------------------------------------------------- oracle sample (CPU)
+def oracle_sample(w, host_inp, seconds: float, rows_hint=None):
+    """Run the fp64 oracle (score row -> budget -> select -> attention row) on
+    (query head, query block) rows of the workload until `seconds` of CPU work
+    are done.  Returns (flops, seconds, rows)."""
+    import numpy as np
+    from block_sparse_attention_stem_b200 import inputs as I
+    from oracle import stem_oracle as O
+
+    p = O.Params(**w.params())
+    L = w.seqlens[0]
+    nb = math.ceil(L / 128)
+    G = w.num_q_heads // w.num_kv_heads
+    heads = sorted({h for h in (0, G, 2 * G + 1) if h < w.num_q_heads})
+    order = rows_hint or [(h, i) for i in list(range(nb - 1, -1, -max(1, nb // 16))) for h in heads]
+    cache = {}
+
+    def head(h):
+        if h not in cache:
+            def sl(t, c):
+                x = t[:L, c:c + 1].contiguous()
+                if w.dtype == "bf16":
+                    return O.dequant(I.raw_bits(x), "bf16")
+                sc = host_inp[{"q": "q_scale", "k": "k_scale", "v": "v_scale"}[n]][c:c + 1].numpy()
+                return O.dequant(I.raw_bits(x), "fp8", sc)
+            hk = h // G
+            n = "q"; qh = sl(host_inp["q"], h)
+            n = "k"; kh = sl(host_inp["k"], hk)
+            n = "v"; vh = sl(host_inp["v"], hk)
+            cache[h] = (qh, kh, vh)
+        return cache[h]
+
+    flops = 0.0
+    spent = 0.0
+    done = []
+    for (h, i) in order:
+        qh, kh, vh = head(h)
+        t0 = time.perf_counter()
+        srow = O.block_score_row(qh, kh, vh, i, p)
+        b = O.tpd_budget(i, nb, p)
+        sel = O.select_row(srow, i, b, p.sink_blocks, p.window_blocks)
+        rp = np.zeros(nb + 1, dtype=np.int64)
+        rp[i + 1:] = len(sel)
+        O.bsa(qh, kh, vh, [0, L], rp, np.array(sel), p, rows_subset=[(0, i)])
+        spent += time.perf_counter() - t0
+        qi = min(128, L - 128 * i)
+        flops += (i + 1) * (128 // p.stride) ** 2 * 2 * p.stride * 128  # scoring of the row
+        flops += 4 * 128 * ((len(sel) - 1) * qi * 128 + qi * (qi + 1) / 2)  # attention of the row
+        done.append((h, i))
+        if spent >= seconds:
+            break
+    return flops, spent, done
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [x.get("num_threads") for x in threadpool_info() if x.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:  # noqa: BLE001
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+# ---------------------------------------------------------------- our implementation
+def run_ours(args):
+    import torch
+
+    rank, world, local = dist_env()
+    if world > 1:
+        torch.cuda.set_device(local)
+    dist_init("nccl" if world > 1 else "gloo")
+    dev = torch.device("cuda", torch.cuda.current_device())
+
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+
+    w = I.workload(args.workload)
+    seed = w.seed + 1000 * rank  # independent layer per rank
+    inp = I.make_inputs(w, seed=seed, device="cuda")
+    torch.cuda.synchronize()
+    qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w.cu_seqlens(), q_scale=inp["q_scale"], k_scale=inp["k_scale"],
+                     v_scale=inp["v_scale"], cu_seqlens_dev=inp["cu_seqlens"])
+    params = b.make_params(**w.params())
+    pl = b.stem_plan(qkv, params)
+    T, hq, hkv = w.total_tokens, w.num_q_heads, w.num_kv_heads
+    scores = torch.empty(hq, pl.nb_total, pl.nb_max, dtype=torch.float32, device=dev)
+    vbonus = torch.empty(hkv, pl.nb_total, dtype=torch.float32, device=dev)
+    budgets = torch.empty(pl.num_rows, dtype=torch.int32, device=dev)
+    row_ptr = torch.empty(pl.num_rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(pl.nnz, dtype=torch.int32, device=dev)
+    out = torch.empty(T, hq, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    ws = torch.empty(pl.ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(ev):
+        ev[0].record(stream)
+        b.stem_score(qkv, params, scores, vbonus, ws, stream)
+        ev[1].record(stream)
+        b.stem_select(qkv, params, scores, budgets, row_ptr, col_idx, ws, stream)
+        ev[2].record(stream)
+        b.stem_bsa_fwd(qkv, params, row_ptr, col_idx, out, lse, ws, stream)
+        ev[3].record(stream)
+
+    mk = lambda: [torch.cuda.Event(enable_timing=True) for _ in range(4)]  # noqa: E731
+    for _ in range(args.warmup):
+        step(mk())
+    torch.cuda.synchronize()
+    status = b.stem_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after warm-up: {b.stem_status_string(status)}")
+
+    sampler = ClockSampler(gpu_device_id(torch))
+    evs = [mk() for _ in range(args.steps)]
+    dist_barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.25)  # let the sampler take its first reading
+    for k in range(args.steps):
+        step(evs[k])
+    torch.cuda.synchronize()
+    dist_barrier()
+    clocks = sampler.stop()
+    status = b.stem_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status after timing: {b.stem_status_string(status)}")
+
+    total_ms = evs[0][0].elapsed_time(evs[-1][3])
+    score_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / args.steps
+    select_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / args.steps
+    bsa_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / args.steps
+    step_ms_local = total_ms / args.steps
+    step_ms = dist_max(step_ms_local, device=dev)
+    flops_rank = pl.score_flops + pl.attn_flops
+    flops_all = dist_sum(flops_rank, device=dev)
+    value = flops_all / (step_ms * 1e-3) / 1e12
+
+    # dense comparator: the same attention kernel with every causal block listed
+    dense_rows = torch.arange(pl.num_rows, dtype=torch.int64)
+    nb = pl.nb_total
+    i_of_row = dense_rows % nb  # one sequence
+    counts = (i_of_row + 1).to(torch.int32)
+    drp = torch.zeros(pl.num_rows + 1, dtype=torch.int32)
+    drp[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    dci = torch.cat([torch.arange(int(c), dtype=torch.int32) for c in counts[:nb]]).repeat(hq)
+    drp, dci = drp.to(dev), dci.to(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    b.stem_bsa_fwd(qkv, params, drp, dci, out, lse, ws, stream)
+    e0.record(stream)
+    nd = 3
+    for _ in range(nd):
+        b.stem_bsa_fwd(qkv, params, drp, dci, out, lse, ws, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    dense_ms = e0.elapsed_time(e1) / nd
+    del drp, dci
+
+    # end to end through the public API with host buffers: H2D inputs, one
+    # stem_prefill call, D2H of the result, every step
+    e2e = None
+    if not args.no_e2e:
+        hq_t = inp["q"].cpu().pin_memory()
+        hk_t = inp["k"].cpu().pin_memory()
+        hv_t = inp["v"].cpu().pin_memory()
+        h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        h_lse = torch.empty(lse.shape, dtype=lse.dtype).pin_memory()
+        pws = torch.empty(pl.ws_prefill_bytes, dtype=torch.uint8, device=dev)
+        dq, dk, dv = torch.empty_like(inp["q"]), torch.empty_like(inp["k"]), torch.empty_like(inp["v"])
+        qkv2 = b.make_qkv(dq, dk, dv, w.cu_seqlens(), q_scale=inp["q_scale"], k_scale=inp["k_scale"],
+                          v_scale=inp["v_scale"], cu_seqlens_dev=inp["cu_seqlens"])
+
+        def e2e_step():
+            dq.copy_(hq_t, non_blocking=True)
+            dk.copy_(hk_t, non_blocking=True)
+            dv.copy_(hv_t, non_blocking=True)
+            b.stem_prefill(qkv2, params, out, lse, None, None, pws, stream, return_lists=False)
+            h_out.copy_(out, non_blocking=True)
+            h_lse.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        ke = max(2, min(args.steps, 5))
+        dist_barrier()
+        a0, a1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a0.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        a1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = dist_max(a0.elapsed_time(a1) / ke, device=dev)
+        e2e = {"value": round(flops_all / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+               "ms_per_step": round(e2e_ms, 3),
+               "h2d_bytes_per_step": int(hq_t.numel() * hq_t.element_size() + hk_t.numel() * hk_t.element_size()
+                                         + hv_t.numel() * hv_t.element_size()),
+               "d2h_bytes_per_step": int(h_out.numel() * h_out.element_size() + h_lse.numel() * 4),
+               "steps": ke, "api": "stem_prefill"}
+        del pws, dq, dk, dv
+
+    peaks, peak_kind = load_peaks()
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    if w.dtype == "fp8":
+        peak *= 2.0  # nominal fp8 : bf16 dense ratio
+    achieved = pl.attn_flops / (bsa_ms * 1e-3) / 1e12
+    traffic = bsa_traffic_per_launch() if w.dtype == "bf16" else None
+    roofline = {"bound": "tensor", "kernel": "bsa_kernel", "achieved": round(achieved, 2), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
+                "peak_source": f"{peak_kind} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if w.dtype == "fp8"
+                                                                      else "") + " of MEASURED_PEAKS.json",
+                "flops_per_launch": pl.attn_flops, "ms_per_launch": round(bsa_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        host = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+        fl, sec, rows = oracle_sample(w, host, args.cpu_seconds)
+        cpu = {"value": round(fl / sec / 1e12, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+               "sample": (f"{len(rows)} (query head, query block) rows of this workload, longest blocks first "
+                          f"(first {rows[:3]}...): fp64 block-score row, budget, top-k, attention row; "
+                          f"{sec:.1f} s, {fl / 1e9:.1f} GFLOP")}
+
+    launches_per_step = 5 * math.ceil(len([L for L in w.seqlens if L > 0]) / 8)
+    res = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(step_ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic (seeded, device RNG)",
+        "config": describe(w),
+        "stages_ms": {"score": round(score_ms, 3), "select": round(select_ms, 3), "bsa": round(bsa_ms, 3)},
+        "dense_bsa_ms": round(dense_ms, 3), "speedup_vs_dense": round(dense_ms / step_ms, 3),
+        "density_blocks": round(pl.nnz_per_head / sum(
+            math.ceil(L / 128) * (math.ceil(L / 128) + 1) / 2 for L in w.seqlens), 4),
+        "attn_tflops_selected": round(achieved, 2),
+        "dense_equiv_tflops": round(pl.dense_attn_flops / (step_ms * 1e-3) / 1e12, 2),
+        "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "clocks": clocks,
+        "gpu_launches": launches_per_step * args.steps,
+    }
+    dist_barrier()
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+    dist_done()
+
+
+# ---------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    import torch
+    from block_sparse_attention_stem_b200 import inputs as I
+
+    w = I.workload(args.workload)
+    inp = I.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+    host = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
+    per_step = max(2.0, min(args.cpu_seconds, 20.0))
+    for _ in range(args.warmup):
+        oracle_sample(w, host, per_step / 4)
+    fl_tot, sec_tot, rows_tot = 0.0, 0.0, 0
+    for _ in range(args.steps):
+        fl, sec, rows = oracle_sample(w, host, per_step)
+        fl_tot += fl
+        sec_tot += sec
+        rows_tot += len(rows)
+    value = fl_tot / sec_tot / 1e12
+    ms = sec_tot / args.steps * 1e3
+    res = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 1), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, device RNG)",
+        "config": describe(w),
+        "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                         "sample": f"{rows_tot} (query head, query block) rows over {args.steps} steps, "
+                                   f"about {per_step:.0f} s each"},
+        "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,97 @@
+// k_vnorm.cu — value-magnitude bonus of the output-aware metric.
+//
+// "Stem" (gist.science zh summary §2.2; de summary §2 B): the metric adds
+// beta * max(0, log ||V_j||^2); the value norms are max-pooled per key block.
+//   vbonus[hk][g0 + j] = beta * max(0, ln max_{t in block j} ||v_t||^2)
+//
+// One CTA per key block reads the block's 128 tokens x Hkv heads x 128 values
+// (256 KB bf16, contiguous in the packed [T, Hkv, d] layout) once with 16-byte
+// loads; 8 lanes cover one (token, head) row of 128 values.  HBM-bound.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+
+#include "stem_device.cuh"
+#include "stem_kernels.h"
+
+namespace stem {
+
+template <bool kFp8>
+__global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const uint8_t* __restrict__ v,
+                                                    const float* __restrict__ v_scale, int hkv, int nbtot,
+                                                    float beta, float* __restrict__ vbonus) {
+  extern __shared__ unsigned int s_max[];  // [hkv] bit patterns of non-negative floats
+  const int s = find_seq(batch, blockIdx.x);
+  const int j = blockIdx.x - batch.item0[s];
+  const int t0 = j * kBlock;
+  const int ntok = min(kBlock, batch.len[s] - t0);
+  for (int h = threadIdx.x; h < hkv; h += blockDim.x) s_max[h] = 0u;
+  __syncthreads();
+
+  constexpr int kElt = kFp8 ? 1 : 2;
+  constexpr int kLanesPerRow = (kHeadDim * kElt) / 16;  // 16-byte vectors per row: 16 (bf16) or 8 (fp8)
+  const int rows = ntok * hkv;
+  const int sub = threadIdx.x % kLanesPerRow;
+  const int row_step = blockDim.x / kLanesPerRow;
+  const uint8_t* base = v + (static_cast<size_t>(batch.tok0[s]) + t0) * hkv * kHeadDim * kElt;
+  for (int r0 = threadIdx.x / kLanesPerRow; r0 - static_cast<int>(threadIdx.x / kLanesPerRow) < rows;
+       r0 += row_step) {
+    float acc = 0.f;
+    const bool valid = r0 < rows;
+    if (valid) {
+      const uint4 w = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(r0) * kHeadDim * kElt + sub * 16);
+      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+      if constexpr (!kFp8) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float lo = __uint_as_float(u[q] << 16);
+          const float hi = __uint_as_float(u[q] & 0xFFFF0000u);
+          acc = fmaf(lo, lo, acc);
+          acc = fmaf(hi, hi, acc);
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int b = 0; b < 4; b += 2) {
+            const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((u[q] >> (8 * b)) & 0xFFFFu);
+            const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
+            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            acc = fmaf(f.x, f.x, acc);
+            acc = fmaf(f.y, f.y, acc);
+          }
+        }
+      }
+    }
+    // reduce over the lanes of this row
+#pragma unroll
+    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (valid && sub == 0) {
+      const int h = r0 % hkv;
+      if constexpr (kFp8) acc *= v_scale[h] * v_scale[h];
+      atomicMax(&s_max[h], __float_as_uint(acc));
+    }
+  }
+  __syncthreads();
+  const int g = batch.g0[s] + j;
+  for (int h = threadIdx.x; h < hkv; h += blockDim.x) {
+    const float m = __uint_as_float(s_max[h]);
+    const float lg = logf(m);  // ln 0 = -inf -> bonus 0
+    vbonus[static_cast<size_t>(h) * nbtot + g] = beta * fmaxf(0.f, lg);
+  }
+}
+
+cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv,
+                         int nbtot, float beta, float* vbonus, cudaStream_t stream) {
+  const int items = batch.item0[batch.n];
+  if (items == 0) return cudaSuccess;
+  const size_t smem = sizeof(unsigned int) * static_cast<size_t>(hkv);
+  if (fp8)
+    vnorm_kernel<true><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, nbtot,
+                                                     beta, vbonus);
+  else
+    vnorm_kernel<false><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, nbtot,
+                                                      beta, vbonus);
+  return cudaGetLastError();
+}
+
+}  // namespace stem

@@ -1,0 +1,393 @@
+// stem_api.cu — the C ABI of include/stem.h: argument validation, planning
+// (sizes, nnz, work counts), per-sequence launch batches, TMA descriptor
+// encoding and kernel launches.  No allocation, no host<->device copies in
+// the compute calls, no synchronisation.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstring>
+#include <vector>
+
+#include "stem.h"
+#include "stem_internal.h"
+#include "stem_kernels.h"
+
+using namespace stem;
+
+namespace {
+
+constexpr size_t kStatusBytes = 256;
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct SeqInfo {
+  int idx;      // sequence number
+  int32_t tok0, len, nb, g0;
+  int64_t csr0; // CSR base of the sequence inside one head
+};
+
+struct Plan {
+  stem_plan_t pub;
+  std::vector<SeqInfo> seqs;  // non-empty sequences, longest first
+  size_t off_vbonus, off_scores, off_budgets, off_rowptr, off_colidx;
+};
+
+stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
+  if (!qkv || !p) return STEM_ERR_INVALID_ARG;
+  if (qkv->dtype != STEM_BF16 && qkv->dtype != STEM_FP8_E4M3) return STEM_ERR_INVALID_ARG;
+  if (qkv->num_seqs < 1 || !qkv->cu_seqlens_host || qkv->total_tokens < 0) return STEM_ERR_INVALID_ARG;
+  if (qkv->num_q_heads < 1 || qkv->num_kv_heads < 1 || qkv->num_q_heads % qkv->num_kv_heads != 0)
+    return STEM_ERR_INVALID_ARG;
+  if (qkv->head_dim != kHeadDim) return qkv->head_dim < 1 ? STEM_ERR_INVALID_ARG : STEM_ERR_UNSUPPORTED;
+  const int32_t* cu = qkv->cu_seqlens_host;
+  if (cu[0] != 0) return STEM_ERR_INVALID_ARG;
+  for (int s = 0; s < qkv->num_seqs; ++s)
+    if (cu[s + 1] < cu[s]) return STEM_ERR_INVALID_ARG;
+  if (cu[qkv->num_seqs] != qkv->total_tokens) return STEM_ERR_INVALID_ARG;
+  if (p->block_size != kBlock) return p->block_size < 1 ? STEM_ERR_INVALID_ARG : STEM_ERR_UNSUPPORTED;
+  if (p->stride < 1 || kBlock % p->stride != 0) return STEM_ERR_INVALID_ARG;
+  if (p->stride != 4 && p->stride != 8) return STEM_ERR_UNSUPPORTED;
+  if (p->chunk_size < 1) return STEM_ERR_INVALID_ARG;
+  if (!(p->norm > 0.0) || !std::isfinite(p->norm)) return STEM_ERR_INVALID_ARG;
+  if (!(p->beta >= 0.0) || !std::isfinite(p->beta)) return STEM_ERR_INVALID_ARG;
+  if (!(p->keep_ratio > 0.0 && p->keep_ratio <= 1.0)) return STEM_ERR_INVALID_ARG;
+  if (!(p->mu > 0.0 && p->mu <= 1.0)) return STEM_ERR_INVALID_ARG;
+  if (p->sink_blocks < 0 || p->window_blocks < 1) return STEM_ERR_INVALID_ARG;
+  if (!(p->softmax_scale >= 0.0) || !std::isfinite(p->softmax_scale)) return STEM_ERR_INVALID_ARG;
+  if (p->budget_mode != STEM_BUDGET_RELATIVE && p->budget_mode != STEM_BUDGET_ABSOLUTE) return STEM_ERR_INVALID_ARG;
+  return STEM_OK;
+}
+
+stem_status_t make_plan(const stem_qkv_t* qkv, const stem_params_t* p, Plan* out) {
+  stem_status_t st = validate(qkv, p);
+  if (st != STEM_OK) return st;
+  const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
+  const int s = p->stride, gpb = kBlock / s;
+  Plan pl{};
+  int64_t nbtot = 0, nb_max = 0, nnz_h = 0;
+  double pairs_sel = 0, pairs_dense = 0, score_pairs = 0;
+  for (int q = 0; q < qkv->num_seqs; ++q) {
+    const int32_t o = qkv->cu_seqlens_host[q];
+    const int32_t L = qkv->cu_seqlens_host[q + 1] - o;
+    const int32_t nb = (L + kBlock - 1) / kBlock;
+    if (nb > 0) {
+      SeqInfo si{q, o, L, nb, static_cast<int32_t>(nbtot), nnz_h};
+      for (int i = 0; i < nb; ++i) {
+        const int32_t b = tpd_budget(i, nb, p->keep_ratio, p->mu, p->sink_blocks, p->window_blocks,
+                                     p->budget_mode);
+        nnz_h += b;
+        const double qi = std::min(kBlock, L - i * kBlock);
+        pairs_sel += (b - 1) * qi * kBlock + qi * (qi + 1) / 2;
+        pairs_dense += static_cast<double>(i) * qi * kBlock + qi * (qi + 1) / 2;
+      }
+      score_pairs += static_cast<double>(nb) * (nb + 1) / 2 * gpb * gpb;
+      pl.seqs.push_back(si);
+    }
+    nbtot += nb;
+    nb_max = std::max<int64_t>(nb_max, nb);
+  }
+  if (nb_max == 0) nb_max = 1;
+  const int64_t rows = static_cast<int64_t>(hq) * nbtot;
+  const int64_t nnz = nnz_h * hq;
+  if (nnz > INT32_MAX || rows + 1 > INT32_MAX) return STEM_ERR_UNSUPPORTED;
+  std::stable_sort(pl.seqs.begin(), pl.seqs.end(), [](const SeqInfo& a, const SeqInfo& b) { return a.nb > b.nb; });
+
+  stem_plan_t& pub = pl.pub;
+  pub.nb_total = nbtot;
+  pub.nb_max = nb_max;
+  pub.num_rows = rows;
+  pub.nnz = nnz;
+  pub.nnz_per_head = nnz_h;
+  pub.scores_bytes = static_cast<size_t>(rows) * nb_max * sizeof(float);
+  pub.vbonus_bytes = static_cast<size_t>(hkv) * nbtot * sizeof(float);
+  pl.off_vbonus = kStatusBytes;
+  pub.ws_bytes = pl.off_vbonus + align256(pub.vbonus_bytes);
+  pl.off_scores = pub.ws_bytes;
+  pl.off_budgets = pl.off_scores + align256(pub.scores_bytes);
+  pl.off_rowptr = pl.off_budgets + align256(static_cast<size_t>(rows) * 4);
+  pl.off_colidx = pl.off_rowptr + align256(static_cast<size_t>(rows + 1) * 4);
+  pub.ws_prefill_bytes = pl.off_colidx + align256(static_cast<size_t>(nnz) * 4);
+  pub.attn_flops = 4.0 * kHeadDim * hq * pairs_sel;
+  pub.dense_attn_flops = 4.0 * kHeadDim * hq * pairs_dense;
+  pub.score_flops = 2.0 * s * kHeadDim * hq * score_pairs;
+  *out = std::move(pl);
+  return STEM_OK;
+}
+
+stem_status_t check_tensors(const stem_qkv_t* qkv) {
+  if (qkv->total_tokens > 0) {
+    if (!qkv->q || !qkv->k || !qkv->v || !qkv->cu_seqlens) return STEM_ERR_INVALID_ARG;
+    if (!aligned16(qkv->q) || !aligned16(qkv->k) || !aligned16(qkv->v)) return STEM_ERR_MISALIGNED;
+  }
+  if (qkv->dtype == STEM_FP8_E4M3 && (!qkv->q_scale || !qkv->k_scale || !qkv->v_scale)) return STEM_ERR_INVALID_ARG;
+  return STEM_OK;
+}
+
+// Split the non-empty sequences into launch batches of at most
+// kMaxSeqPerLaunch; items(si) is the number of CTAs a sequence needs.
+template <class F>
+std::vector<SeqBatch> make_batches(const Plan& pl, F items) {
+  std::vector<SeqBatch> out;
+  for (size_t b0 = 0; b0 < pl.seqs.size(); b0 += kMaxSeqPerLaunch) {
+    SeqBatch b{};
+    b.n = static_cast<int32_t>(std::min<size_t>(kMaxSeqPerLaunch, pl.seqs.size() - b0));
+    b.item0[0] = 0;
+    for (int q = 0; q < b.n; ++q) {
+      const SeqInfo& si = pl.seqs[b0 + q];
+      b.tok0[q] = si.tok0;
+      b.len[q] = si.len;
+      b.nb[q] = si.nb;
+      b.g0[q] = si.g0;
+      b.csr0[q] = si.csr0;
+      b.item0[q + 1] = b.item0[q] + items(si);
+    }
+    for (int q = b.n; q < kMaxSeqPerLaunch; ++q) b.item0[q + 1] = b.item0[q];
+    out.push_back(b);
+  }
+  return out;
+}
+
+// ---------------------------------------------------------------- TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &ptr, 12000, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 3-D map over one sequence of a [T, H, 128] tensor: dims (d, head, token),
+// box (inner, 1, box_tokens) traversed with token stride `tstride`, 128-B swizzle.
+bool encode_seq_map(CUtensorMap* m, const void* base, bool fp8, int heads, int tok0, int len, int box_tokens,
+                    int tstride) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const size_t elt = fp8 ? 1 : 2;
+  const uint8_t* b = static_cast<const uint8_t*>(base) + static_cast<size_t>(tok0) * heads * kHeadDim * elt;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(len)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(kHeadDim * elt), static_cast<cuuint64_t>(heads * kHeadDim * elt)};
+  cuuint32_t box[3] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), 1u, static_cast<cuuint32_t>(box_tokens)};
+  cuuint32_t estr[3] = {1u, 1u, static_cast<cuuint32_t>(tstride)};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3,
+                  const_cast<uint8_t*>(b), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+stem_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? STEM_OK : STEM_ERR_CUDA; }
+
+double sm_scale(const stem_params_t* p) {
+  return p->softmax_scale > 0.0 ? p->softmax_scale : 1.0 / std::sqrt(static_cast<double>(kHeadDim));
+}
+
+// ---------------------------------------------------------------- stages
+stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, float* scores,
+                        float* vbonus, int* status, cudaStream_t stream) {
+  const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
+  const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads, s = p->stride;
+  const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
+  for (const SeqBatch& b : make_batches(pl, [](const SeqInfo& si) { return si.nb; })) {
+    stem_status_t st = cuda_status(
+        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, nbtot, static_cast<float>(p->beta), vbonus, stream));
+    if (st != STEM_OK) return st;
+  }
+  ScoreArgs a{};
+  a.hq = hq;
+  a.hkv = hkv;
+  a.nbtot = nbtot;
+  a.nb_max = nb_max;
+  a.stride = s;
+  a.scale = static_cast<float>(1.0 / (std::sqrt(static_cast<double>(kHeadDim)) * s * p->norm));
+  a.q_scale = qkv->q_scale;
+  a.k_scale = qkv->k_scale;
+  a.vbonus = vbonus;
+  a.scores = scores;
+  a.status = status;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * ((si.nb + s - 1) / s); })) {
+    ScoreMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    for (int q = 0; q < b.n; ++q) {
+      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], 256, s) ||
+          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], 256, s))
+        return STEM_ERR_CUDA;
+    }
+    stem_status_t st = cuda_status(launch_score(maps, b, a, fp8, stream));
+    if (st != STEM_OK) return st;
+  }
+  return STEM_OK;
+}
+
+stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, const float* scores,
+                         int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, cudaStream_t stream) {
+  const int hq = qkv->num_q_heads;
+  const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
+  for (const SeqBatch& b : make_batches(pl, [](const SeqInfo&) { return 1; })) {
+    stem_status_t st = cuda_status(launch_budget(b, hq, nbtot, pl.pub.nnz_per_head, p->keep_ratio, p->mu,
+                                                 p->sink_blocks, p->window_blocks, p->budget_mode, budgets,
+                                                 row_ptr, stream));
+    if (st != STEM_OK) return st;
+  }
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
+    stem_status_t st = cuda_status(launch_select(b, hq, nbtot, nb_max, p->sink_blocks, p->window_blocks, scores,
+                                                 budgets, row_ptr, col_idx, stream));
+    if (st != STEM_OK) return st;
+  }
+  return STEM_OK;
+}
+
+stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, const int32_t* row_ptr,
+                      const int32_t* col_idx, void* out, float* lse, int* status, cudaStream_t stream) {
+  const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
+  const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
+  BsaArgs a{};
+  a.hq = hq;
+  a.hkv = hkv;
+  a.nbtot = static_cast<int>(pl.pub.nb_total);
+  a.total_tokens = qkv->total_tokens;
+  a.scale_log2 = static_cast<float>(sm_scale(p) * 1.4426950408889634);
+  a.q_scale = qkv->q_scale;
+  a.k_scale = qkv->k_scale;
+  a.v_scale = qkv->v_scale;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
+  a.out = out;
+  a.lse = lse;
+  a.status = status;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
+    BsaMaps maps;
+    std::memset(&maps, 0, sizeof(maps));
+    for (int q = 0; q < b.n; ++q) {
+      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1) ||
+          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
+          !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1))
+        return STEM_ERR_CUDA;
+    }
+    stem_status_t st = cuda_status(launch_bsa(maps, b, a, fp8, stream));
+    if (st != STEM_OK) return st;
+  }
+  return STEM_OK;
+}
+
+stem_status_t clear_status(void* ws, cudaStream_t stream) {
+  return cuda_status(cudaMemsetAsync(ws, 0, sizeof(int), stream));
+}
+
+}  // namespace
+
+extern "C" {
+
+stem_status_t stem_plan(const stem_qkv_t* qkv, const stem_params_t* params, stem_plan_t* out) {
+  if (!out) return STEM_ERR_INVALID_ARG;
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st == STEM_OK) *out = pl.pub;
+  return st;
+}
+
+stem_status_t stem_score(const stem_qkv_t* qkv, const stem_params_t* params, float* scores, float* vbonus,
+                         void* ws, size_t ws_bytes, stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if ((st = check_tensors(qkv)) != STEM_OK) return st;
+  if (!scores || !ws) return STEM_ERR_INVALID_ARG;
+  if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  float* vb = vbonus ? vbonus : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_vbonus);
+  return run_score(qkv, params, pl, scores, vb, static_cast<int*>(ws), s);
+}
+
+stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params, const float* scores,
+                          int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
+                          stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if (!scores || !budgets || !row_ptr || !ws || (!col_idx && pl.pub.nnz > 0)) return STEM_ERR_INVALID_ARG;
+  if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  return run_select(qkv, params, pl, scores, budgets, row_ptr, col_idx, s);
+}
+
+stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params, const int32_t* row_ptr,
+                           const int32_t* col_idx, void* out, float* lse, void* ws, size_t ws_bytes,
+                           stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if ((st = check_tensors(qkv)) != STEM_OK) return st;
+  if (!row_ptr || !col_idx || !out || !lse || !ws) return STEM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return STEM_ERR_MISALIGNED;
+  if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  return run_bsa(qkv, params, pl, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s);
+}
+
+stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, void* out, float* lse,
+                           int32_t* row_ptr_out, int32_t* col_idx_out, void* ws, size_t ws_bytes,
+                           stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if ((st = check_tensors(qkv)) != STEM_OK) return st;
+  if (!out || !lse || !ws) return STEM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return STEM_ERR_MISALIGNED;
+  if (ws_bytes < pl.pub.ws_prefill_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  float* vbonus = reinterpret_cast<float*>(w + pl.off_vbonus);
+  float* scores = reinterpret_cast<float*>(w + pl.off_scores);
+  int32_t* budgets = reinterpret_cast<int32_t*>(w + pl.off_budgets);
+  int32_t* row_ptr = row_ptr_out ? row_ptr_out : reinterpret_cast<int32_t*>(w + pl.off_rowptr);
+  int32_t* col_idx = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(w + pl.off_colidx);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  if ((st = run_score(qkv, params, pl, scores, vbonus, status, s)) != STEM_OK) return st;
+  if ((st = run_select(qkv, params, pl, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
+  return run_bsa(qkv, params, pl, row_ptr, col_idx, out, lse, status, s);
+}
+
+stem_status_t stem_read_device_status(const void* ws, stem_stream_t stream, stem_status_t* out) {
+  if (!ws || !out) return STEM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return STEM_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return STEM_ERR_CUDA;
+  *out = static_cast<stem_status_t>(v);
+  return STEM_OK;
+}
+
+const char* stem_status_string(stem_status_t status) {
+  switch (status) {
+    case STEM_OK: return "ok";
+    case STEM_ERR_INVALID_ARG: return "invalid argument";
+    case STEM_ERR_UNSUPPORTED: return "unsupported configuration";
+    case STEM_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+    case STEM_ERR_MISALIGNED: return "tensor pointer not 16-byte aligned";
+    case STEM_ERR_CUDA: return "CUDA error";
+    case STEM_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case STEM_ERR_BAD_BLOCKLIST: return "malformed block list entry skipped";
+  }
+  return "unknown status";
+}
+
+int32_t stem_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,64 @@
+// stem_kernels.h — kernel launch interfaces used by the host API (stem_api.cu).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "stem_internal.h"
+
+namespace stem {
+
+// Per-sequence TMA descriptors of one launch (kernel parameters, so the
+// kernels need no descriptor copies in global memory).
+struct ScoreMaps {
+  CUtensorMap q[kMaxSeqPerLaunch];  // token traversal stride s, box 256 tokens
+  CUtensorMap k[kMaxSeqPerLaunch];
+};
+
+struct BsaMaps {
+  CUtensorMap q[kMaxSeqPerLaunch];  // box 128 tokens
+  CUtensorMap k[kMaxSeqPerLaunch];
+  CUtensorMap v[kMaxSeqPerLaunch];
+};
+
+struct ScoreArgs {
+  int hq, hkv, nbtot, nb_max, stride;
+  float scale;              // 1 / (sqrt(d) s n)
+  const float* q_scale;     // fp8 only
+  const float* k_scale;
+  const float* vbonus;      // [Hkv][NBtot]
+  float* scores;            // [Hq][NBtot][nb_max]
+  int* status;
+};
+
+struct BsaArgs {
+  int hq, hkv, nbtot, total_tokens;
+  float scale_log2;         // softmax scale * log2(e)
+  const float* q_scale;     // fp8 only
+  const float* k_scale;
+  const float* v_scale;
+  const int32_t* row_ptr;
+  const int32_t* col_idx;
+  void* out;                // bf16 [T, Hq, d]
+  float* lse;               // [Hq][T]
+  int* status;
+};
+
+cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int nbtot,
+                         float beta, float* vbonus, cudaStream_t stream);
+cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args, bool fp8,
+                         cudaStream_t stream);
+cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_per_head, double rho, double mu,
+                          int sink, int window, int mode, int32_t* budgets, int32_t* row_ptr, cudaStream_t stream);
+cudaError_t launch_select(const SeqBatch& batch, int hq, int nbtot, int nb_max, int sink, int window,
+                          const float* scores, const int32_t* budgets, const int32_t* row_ptr, int32_t* col_idx,
+                          cudaStream_t stream);
+cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
+                       cudaStream_t stream);
+
+size_t score_smem_bytes();
+size_t bsa_smem_bytes(bool fp8);
+
+}  // namespace stem

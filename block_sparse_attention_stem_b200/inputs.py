@@ -96,10 +96,11 @@ def fp8_layer_mu(layer: int) -> float:
 
 def _draw(w: Workload, gen: torch.Generator):
     T, hq, hkv, d = w.total_tokens, w.num_q_heads, w.num_kv_heads, w.head_dim
-    q = torch.randn(T, hq, d, generator=gen, dtype=torch.float32)
-    k = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32)
-    v = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32)
-    v *= torch.exp(0.5 * torch.randn(T, hkv, 1, generator=gen, dtype=torch.float32))
+    dev = gen.device
+    q = torch.randn(T, hq, d, generator=gen, dtype=torch.float32, device=dev)
+    k = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32, device=dev)
+    v = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32, device=dev)
+    v *= torch.exp(0.5 * torch.randn(T, hkv, 1, generator=gen, dtype=torch.float32, device=dev))
     if w.sink_boost:
         G = hq // hkv
         cu = w.cu_seqlens()
@@ -120,12 +121,14 @@ def _to_fp8(x: torch.Tensor):
     return x8.view(torch.uint8), scale
 
 
-def make_inputs(w: Workload, seed: int | None = None) -> dict:
-    """CPU tensors: q [T,Hq,d], k/v [T,Hkv,d] as bf16 (or uint8 e4m3 bytes with
-    fp32 per-head scales q_scale/k_scale/v_scale), plus cu_seqlens int32."""
-    gen = torch.Generator("cpu").manual_seed(w.seed if seed is None else seed)
+def make_inputs(w: Workload, seed: int | None = None, device: str = "cpu") -> dict:
+    """q [T,Hq,d], k/v [T,Hkv,d] as bf16 (or uint8 e4m3 bytes with fp32
+    per-head scales q_scale/k_scale/v_scale), plus cu_seqlens int32, drawn on
+    `device` with that device's generator (the CPU stream is the reference one
+    the tests use; a CUDA generator gives the same distributions faster)."""
+    gen = torch.Generator(device).manual_seed(w.seed if seed is None else seed)
     q, k, v = _draw(w, gen)
-    out = dict(cu_seqlens=torch.tensor(w.cu_seqlens(), dtype=torch.int32))
+    out = dict(cu_seqlens=torch.tensor(w.cu_seqlens(), dtype=torch.int32, device=device))
     if w.dtype == "bf16":
         out.update(q=q.to(torch.bfloat16), k=k.to(torch.bfloat16), v=v.to(torch.bfloat16),
                    q_scale=None, k_scale=None, v_scale=None)

@@ -1,0 +1,203 @@
+/*
+ * stem.h — C ABI of the Stem long-context prefill hot path on NVIDIA B200 (sm_100a).
+ *
+ * The method (sources are cited by page title and section):
+ *  - "Stem: Rethinking Causal Information Flow in Sparse Attention", AngelSlim
+ *    documentation (stem.md), §2.1 Block-Level Scoring, §2.2 Top-k Schedule,
+ *    §2.3 Block-Sparse Attention, §6 parameter table.
+ *  - the same paper's gist.science summaries (zh §2.1 TPD, §2.2 OAM, §2.3 flow;
+ *    de §2 Methodik A/B/C).
+ *  - the youleyou article on Stem and the HPC-BSA operator, §2.2 (log form of
+ *    the metric) and §3.1 (skip decisions made outside the inner loop; skipped
+ *    blocks are equivalent to -inf scores).
+ *
+ * Pipeline: stem_prefill = stem_score (value-norm bonus + anti-diagonal
+ * downsampled scoring + block max-pool) -> stem_select (token position-decay
+ * budget + top-k with sink and window blocks, emitted as CSR block lists) ->
+ * stem_bsa_fwd (causal block-sparse flash attention over the listed blocks).
+ *
+ * Conventions common to every entry point:
+ *  - All tensor pointers are DEVICE pointers unless the name ends in _host.
+ *  - The library allocates nothing.  The caller owns every buffer, including
+ *    the workspace `ws`, whose size stem_plan() reports.
+ *  - Every compute call is asynchronous on `stream` (a cudaStream_t; NULL is
+ *    the legacy default stream) and performs no host<->device copy and no
+ *    host synchronisation.
+ *  - Argument errors are detected on the host and returned before anything is
+ *    enqueued.  Errors the GPU detects (a malformed block list, a pipeline
+ *    wait that ran out) are written to a status word inside `ws`; read it with
+ *    stem_read_device_status().  Each compute call clears that word first.
+ *  - Tensors: q [T, Hq, d], k and v [T, Hkv, d], d contiguous, rows of all
+ *    sequences packed back to back (cu_seqlens), every base pointer 16-byte
+ *    aligned.  d must be 128 and Hq a multiple of Hkv (grouped-query attention:
+ *    query head h reads KV head h / (Hq/Hkv)).
+ *  - Blocks: each sequence is cut into NB_s = ceil(L_s / 128) blocks of 128
+ *    tokens (the last one may be partial).  Global block index g runs over
+ *    the blocks of sequence 0, then sequence 1, ...; NBtot = sum NB_s and
+ *    nb_max = max NB_s.  Row r = h * NBtot + g of every per-row array belongs
+ *    to query head h and query block g.
+ */
+#ifndef STEM_H
+#define STEM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define STEM_API __attribute__((visibility("default")))
+#else
+#define STEM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so the header needs no CUDA include. */
+typedef struct CUstream_st* stem_stream_t;
+
+typedef enum {
+  STEM_OK = 0,
+  STEM_ERR_INVALID_ARG = 1,          /* a size, parameter or pointer is out of its documented range */
+  STEM_ERR_UNSUPPORTED = 2,          /* valid but not implemented here (e.g. head_dim != 128) */
+  STEM_ERR_WORKSPACE_TOO_SMALL = 3,  /* ws_bytes below what stem_plan() reported for this call */
+  STEM_ERR_MISALIGNED = 4,           /* a tensor base pointer is not 16-byte aligned */
+  STEM_ERR_CUDA = 5,                 /* a CUDA runtime/driver call failed (launch, tensor-map encode) */
+  STEM_ERR_TIMEOUT = 6,              /* device: a pipeline wait exceeded its bound; outputs are invalid */
+  STEM_ERR_BAD_BLOCKLIST = 7         /* device: a CSR entry was out of range or not strictly ascending;
+                                        the offending entry was skipped */
+} stem_status_t;
+
+typedef enum { STEM_BF16 = 0, STEM_FP8_E4M3 = 1 } stem_dtype_t;
+
+/* How keep_ratio sets k_start of the position-decay budget (the pages leave the
+ * mapping open):
+ *   RELATIVE (default): k_start of query block i is ceil(rho * (i + 1)), i.e. a
+ *            fraction of the i+1 causal key blocks of that row;
+ *   ABSOLUTE: k_start = ceil(rho * NB_s) for every row of the sequence. */
+typedef enum { STEM_BUDGET_RELATIVE = 0, STEM_BUDGET_ABSOLUTE = 1 } stem_budget_mode_t;
+
+/* Method parameters (AngelSlim documentation §6 defaults in brackets). */
+typedef struct {
+  int32_t block_size;     /* attention block [128]; only 128 is supported */
+  int32_t stride;         /* scoring downsampling stride s [8]; 4 or 8 are supported */
+  int32_t chunk_size;     /* scoring query-chunk width [2048]; > 0; does not change results */
+  double  norm;           /* extra scoring normalisation n [1.0]; > 0 */
+  double  beta;           /* weight of the value-magnitude bonus [0.2]; >= 0 */
+  double  keep_ratio;     /* rho in (0, 1] */
+  double  mu;             /* decay factor (stem_alpha of this layer) in (0, 1] [1.0; 0.7 best] */
+  int32_t sink_blocks;    /* initial blocks always kept [4]; >= 0 */
+  int32_t window_blocks;  /* trailing causal blocks always kept, the diagonal included [4]; >= 1 */
+  double  softmax_scale;  /* attention logit scale; 0 selects 1/sqrt(head_dim) */
+  int32_t budget_mode;    /* stem_budget_mode_t */
+} stem_params_t;
+
+/* Query/key/value description shared by all calls. */
+typedef struct {
+  int32_t dtype;                  /* stem_dtype_t of q, k and v */
+  int32_t num_seqs;               /* >= 1 */
+  int32_t total_tokens;           /* T = cu_seqlens[num_seqs] */
+  const int32_t* cu_seqlens;      /* device [num_seqs + 1], cu[0] = 0, non-decreasing */
+  const int32_t* cu_seqlens_host; /* host copy of the same offsets (used for planning and
+                                     launch geometry; read during the call only) */
+  int32_t num_q_heads;            /* Hq */
+  int32_t num_kv_heads;           /* Hkv, divides Hq */
+  int32_t head_dim;               /* d; must be 128 */
+  const void* q;                  /* [T, Hq, d] bf16 or e4m3 bytes */
+  const void* k;                  /* [T, Hkv, d] */
+  const void* v;                  /* [T, Hkv, d] */
+  const float* q_scale;           /* fp8 only: device [Hq]  dequantisation scales (value = e4m3 * scale) */
+  const float* k_scale;           /* fp8 only: device [Hkv] */
+  const float* v_scale;           /* fp8 only: device [Hkv] */
+} stem_qkv_t;
+
+/* Sizes derived on the host from (cu_seqlens_host, params); data-independent. */
+typedef struct {
+  int64_t nb_total;          /* NBtot */
+  int64_t nb_max;            /* nb_max */
+  int64_t num_rows;          /* Hq * NBtot (length of budgets; row_ptr has num_rows + 1) */
+  int64_t nnz;               /* total listed blocks = sum of the budgets over all rows */
+  int64_t nnz_per_head;      /* nnz / Hq */
+  size_t  scores_bytes;      /* bytes of the fp32 score matrix [Hq][NBtot][nb_max] */
+  size_t  vbonus_bytes;      /* bytes of the fp32 bonus [Hkv][NBtot] */
+  size_t  ws_bytes;          /* workspace for stem_score / stem_select / stem_bsa_fwd */
+  size_t  ws_prefill_bytes;  /* workspace for stem_prefill (holds scores and the CSR) */
+  double  attn_flops;        /* 4 d Hq * (sum over listed blocks of query-key pairs), causal
+                                pairs only on the diagonal block */
+  double  dense_attn_flops;  /* the same with every causal block listed */
+  double  score_flops;       /* 2 * s * d * Hq * (16 x 16 group pairs per causal block pair) */
+} stem_plan_t;
+
+/* Validate (qkv, params) and fill *out.  Host only; touches no device memory
+ * (only cu_seqlens_host is read).  [AngelSlim doc §2.2 / gist-zh §2.1: the
+ * budget k(i) = floor(k_start - k_start (1 - mu) i / N) is data-independent,
+ * so nnz and every size are known before any kernel runs.] */
+STEM_API stem_status_t stem_plan(const stem_qkv_t* qkv, const stem_params_t* params, stem_plan_t* out);
+
+/* Block scores [AngelSlim doc §2.1; gist-zh §2.2 OAM and §2.3 anti-diagonal
+ * downsampling; gist-de §2 C].
+ *   vbonus[hk][g] = beta * max(0, ln max_{t in block g} ||v_t||^2)
+ *   D[h][a][b]    = sum_{u<s} q[a s + u, h] . k[b s + s-1-u, h/G] / (sqrt(d) s n)
+ *   scores[h][g][j] = max over the query groups a of block g and key groups b of
+ *                     block j of D + vbonus[h/G][g0+j]   for j <= i (local index);
+ *                     -inf for i < j < nb_max.
+ * Layout: scores fp32 [Hq][NBtot][nb_max] (row r = h*NBtot+g, column = key block
+ * index local to the sequence); vbonus fp32 [Hkv][NBtot] (may be NULL, then the
+ * workspace holds it).  Groups whose first token is past the sequence end are
+ * ignored; missing tokens of the last group count as zero. */
+STEM_API stem_status_t stem_score(const stem_qkv_t* qkv, const stem_params_t* params,
+                         float* scores, float* vbonus,
+                         void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* Position-decay budgets and top-k block lists [gist-zh §2.1 TPD; AngelSlim doc
+ * §2.2 sink and window blocks; youleyou §3.1 compacted lists].
+ *   c = i + 1, F = {0 .. min(S,c)-1} u {max(0,c-W) .. i}
+ *   k_start = ceil(rho * c) (RELATIVE) or ceil(rho * NB_s) (ABSOLUTE)
+ *   k = floor(k_start - ((k_start * (1 - mu)) * i) / NB_s)   (IEEE fp64, this order)
+ *   b = min(c, max(k, |F|))
+ *   row = F u the b-|F| best other causal blocks by (score desc, index asc),
+ *         NaN ranked as -inf, written in ascending order.
+ * Outputs: budgets int32 [Hq*NBtot], row_ptr int32 [Hq*NBtot + 1] (row_ptr[0] = 0),
+ * col_idx int32 [nnz] (key-block indices local to the sequence). */
+STEM_API stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params,
+                          const float* scores, int32_t* budgets, int32_t* row_ptr,
+                          int32_t* col_idx, void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* Causal block-sparse attention over caller-given CSR lists [gist-zh §2.3 exact
+ * softmax over the chosen blocks only; youleyou §3.1].
+ *   For query token t of block i of row r: keys = union over j in
+ *   col_idx[row_ptr[r] .. row_ptr[r+1]) of the tokens u of block j with u <= t.
+ *   out[t][h] = sum softmax(sigma q_t . k_u) v_u,  lse[h][t] = ln sum exp(sigma q_t . k_u),
+ *   sigma = softmax_scale (or 1/sqrt(d)), times q_scale*k_scale for fp8.
+ * out bf16 [T, Hq, d]; lse fp32 [Hq][T].  Lists must be strictly ascending with
+ * 0 <= j <= i; a violating entry is skipped and STEM_ERR_BAD_BLOCKLIST recorded.
+ * An empty row gives out = 0 and lse = -inf.  fp8: P is rounded to e4m3 for the
+ * P.V product. */
+STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params,
+                           const int32_t* row_ptr, const int32_t* col_idx,
+                           void* out, float* lse,
+                           void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* score -> select -> attention on one stream with no host round trip.
+ * row_ptr_out / col_idx_out may be NULL (the workspace then holds the lists);
+ * ws_bytes >= plan.ws_prefill_bytes. */
+STEM_API stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params,
+                           void* out, float* lse,
+                           int32_t* row_ptr_out, int32_t* col_idx_out,
+                           void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* Synchronise `stream` and read the device status word of `ws` into *out.
+ * Returns STEM_ERR_CUDA if the copy fails. */
+STEM_API stem_status_t stem_read_device_status(const void* ws, stem_stream_t stream, stem_status_t* out);
+
+/* Static string for a status code; never NULL. */
+STEM_API const char* stem_status_string(stem_status_t status);
+
+/* Library version, MAJOR*10000 + MINOR*100 + PATCH. */
+STEM_API int32_t stem_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* STEM_H */

@@ -280,6 +280,24 @@ def block_scores(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens, p: Par
     return S
 
 
+def block_score_row(q: np.ndarray, k: np.ndarray, v: np.ndarray, i: int, p: Params) -> np.ndarray:
+    """Row i of the block-score matrix of ONE sequence and ONE query head:
+    q [L, 1, d], k/v [L, 1, d] fp64 (the query head and its KV head).  Same
+    steps as block_scores, restricted to the query groups of block i and the
+    key groups of blocks 0..i (used to check sampled rows of long inputs)."""
+    B, s = p.block_size, p.stride
+    gpb = B // s
+    L = q.shape[0]
+    ng_valid = cdiv(L, s)
+    a0, a1 = i * gpb, min((i + 1) * gpb, ng_valid)
+    D = downsampled_scores(q, k, s, p.norm, groups=(a0, a1), key_groups=min((i + 1) * gpb, ng_valid))[0]
+    bonus = value_bonus(v[:min((i + 1) * B, L)], [0, min((i + 1) * B, L)], p.beta, B)[0]
+    out = np.empty(i + 1)
+    for j in range(i + 1):
+        out[j] = D[:, j * gpb:min((j + 1) * gpb, ng_valid)].max() + bonus[j]
+    return out
+
+
 # --------------------------------------------------------------------------
 # Step 4: Token Position-Decay budget (gist-zh §2.1 / gist-de §2 A):
 #   k(i) = floor(k_start - k_start * (1 - mu) / N * i),  k_end = mu * k_start,

@@ -1,0 +1,174 @@
+"""GPU parity: the CUDA library (called through its C ABI) against the fp64
+oracle on the same seeded input bytes.
+
+Acceptance (block scores relative 1e-3; budgets and row pointers bit-exact;
+block lists bit-exact except at documented near-ties; attention output within
+2e-2 (bf16) / 6e-2 (fp8) max-abs and LSE within 1e-3, computed with the GPU's
+block lists).
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import stem_oracle as O
+from block_sparse_attention_stem_b200 import inputs as I
+from gpu_common import (check_attention, check_scores, compare_lists, make_gpu_qkv, oparams, oracle_arrays,
+                        to_device)
+
+pytestmark = pytest.mark.gpu
+
+b = pytest.importorskip("block_sparse_attention_stem_b200.binding")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def W(seqlens, hq, hkv, dtype="bf16", seed=10, **kw):
+    base = dict(keep_ratio=0.4, mu=0.7, beta=0.2, sink_blocks=1, window_blocks=2)
+    base.update(kw)
+    return I.Workload(name="case", seqlens=seqlens, num_q_heads=hq, num_kv_heads=hkv, dtype=dtype, seed=seed,
+                      **base)
+
+
+CASES = {
+    "tiny": I.workload("tiny"),
+    "one_block": W([128], 1, 1, keep_ratio=0.5, sink_blocks=1, window_blocks=1),
+    "gqa4_ragged": W([1000], 4, 1, seed=11),
+    "odd_len": W([1001], 2, 2, seed=12, stride=8),
+    "varlen": W([1000, 128, 2088], 8, 2, seed=13, sink_blocks=2, window_blocks=1),
+    "stride4": W([1536], 2, 1, seed=14, stride=4),
+    "multi_tile": W([4096 + 640], 4, 2, seed=15, keep_ratio=0.3, sink_blocks=1, window_blocks=1),
+    "tiny_fp8": I.workload("tiny", dtype="fp8"),
+    "varlen_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=16),
+    "many_seqs": W([128 * (k % 5 + 1) + 8 * k for k in range(11)], 2, 1, seed=17),
+}
+
+
+class Case:
+    """Inputs, GPU results and oracle results of one workload (computed once)."""
+
+    def __init__(self, w):
+        self.w = w
+        self.cu = w.cu_seqlens()
+        self.inp = I.make_inputs(w)
+        self.dinp = to_device(self.inp)
+        self.qkv = make_gpu_qkv(b, self.dinp, self.cu)
+        self.params = b.make_params(**w.params())
+        self.p = oparams(w)
+        self.q, self.k, self.v = oracle_arrays(self.inp, w.dtype)
+        self.ref_scores = O.block_scores(self.q, self.k, self.v, self.cu, self.p)
+        self.ref_bonus = O.value_bonus(self.v, self.cu, self.p.beta)
+
+
+_cache = {}
+
+
+def get_case(name):
+    if name not in _cache:
+        _cache[name] = Case(CASES[name])
+    return _cache[name]
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_scores_and_bonus(name):
+    c = get_case(name)
+    scores, vbonus, ws = b.stem_score(c.qkv, c.params)
+    assert b.stem_read_device_status(ws) == 0
+    check_scores(scores.cpu().numpy().astype(np.float64), c.ref_scores, c.cu)
+    vb = vbonus.cpu().numpy().astype(np.float64)
+    np.testing.assert_allclose(vb, c.ref_bonus, rtol=1e-5, atol=1e-5)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_select_is_bit_exact_on_identical_fp32_scores(name):
+    """Feed the oracle's scores rounded to fp32 to the GPU selection; the oracle
+    selects on the very same fp32 values: budgets, row_ptr and col_idx must be
+    identical (ties resolved by index on both sides)."""
+    c = get_case(name)
+    s32 = c.ref_scores.astype(np.float32)
+    gb, grp, gci, ws = b.stem_select(c.qkv, c.params, torch.from_numpy(s32).cuda())
+    assert b.stem_read_device_status(ws) == 0
+    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p)
+    assert np.array_equal(gb.cpu().numpy(), ob)
+    assert np.array_equal(grp.cpu().numpy(), orp)
+    assert np.array_equal(gci.cpu().numpy(), oci)
+
+
+def test_select_ties_go_to_lowest_index():
+    c = get_case("varlen")
+    rng = np.random.default_rng(3)
+    s32 = np.round(c.ref_scores * 2).astype(np.float32) / 2  # many exact ties
+    s32[rng.random(s32.shape) < 0.05] = np.nan               # NaN ranks as -inf
+    gb, grp, gci, _ = b.stem_select(c.qkv, c.params, torch.from_numpy(s32).cuda())
+    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p)
+    assert np.array_equal(grp.cpu().numpy(), orp)
+    assert np.array_equal(gci.cpu().numpy(), oci)
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_prefill_end_to_end(name):
+    c = get_case(name)
+    out, lse, rp, ci, ws = b.stem_prefill(c.qkv, c.params)
+    assert b.stem_read_device_status(ws) == 0
+    rp, ci = rp.cpu().numpy(), ci.cpu().numpy()
+    ob, orp, oci = O.select(c.ref_scores, c.cu, c.p)
+    compare_lists(rp, ci, orp, oci, c.ref_scores, c.cu, c.w.num_q_heads, c.p.sink_blocks, c.p.window_blocks)
+    # attention with the GPU's own lists
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp, ci, c.p)
+    check_attention(out, lse, ro, rl, c.w.dtype)
+    # stem_prefill == stem_score -> stem_select -> stem_bsa_fwd
+    scores, _, _ = b.stem_score(c.qkv, c.params)
+    _, rp2, ci2, _ = b.stem_select(c.qkv, c.params, scores)
+    assert np.array_equal(rp2.cpu().numpy(), rp) and np.array_equal(ci2.cpu().numpy(), ci)
+    out2, lse2, _ = b.stem_bsa_fwd(c.qkv, c.params, rp2, ci2)
+    assert torch.equal(out2, out) and torch.equal(lse2, lse)
+
+
+@pytest.mark.parametrize("name", ["tiny", "varlen", "varlen_fp8", "multi_tile"])
+def test_dense_comparator_is_causal_attention(name):
+    """Every causal block listed: the result is ordinary causal attention."""
+    c = get_case(name)
+    rp, ci = O.full_csr(c.cu, c.w.num_q_heads)
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, torch.from_numpy(rp.astype(np.int32)).cuda(),
+                                  torch.from_numpy(ci.astype(np.int32)).cuda())
+    assert b.stem_read_device_status(ws) == 0
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp, ci, c.p)
+    check_attention(out, lse, ro, rl, c.w.dtype)
+
+
+def test_malformed_list_entries_are_skipped_and_reported():
+    c = get_case("varlen")
+    rp, ci = O.full_csr(c.cu, c.w.num_q_heads)
+    bad = ci.copy()
+    seqs, nbtot = O.seq_blocks(c.cu)
+    # row of head 1, block 5 of sequence 0: replace its 3rd entry by a block above the diagonal
+    r = 1 * nbtot + 5
+    bad[rp[r] + 2] = 9
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, torch.from_numpy(rp.astype(np.int32)).cuda(),
+                                  torch.from_numpy(bad.astype(np.int32)).cuda())
+    assert b.stem_read_device_status(ws) == 7
+    keep = np.ones(len(ci), dtype=bool)
+    keep[rp[r] + 2] = False
+    rp2 = rp.copy()
+    rp2[r + 1:] -= 1
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp2, ci[keep], c.p)
+    check_attention(out, lse, ro, rl, "bf16")
+
+
+def test_empty_rows_give_zero_output_and_minus_inf_lse():
+    c = get_case("tiny")
+    nrows = 2 * 16
+    rp = torch.zeros(nrows + 1, dtype=torch.int32, device="cuda")
+    ci = torch.zeros(1, dtype=torch.int32, device="cuda")
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, ci)
+    assert b.stem_read_device_status(ws) == 0
+    assert torch.all(out == 0)
+    assert torch.all(torch.isneginf(lse))
+
+
+def test_results_are_deterministic():
+    c = get_case("multi_tile")
+    a = b.stem_prefill(c.qkv, c.params)
+    z = b.stem_prefill(c.qkv, c.params)
+    for x, y in zip(a[:4], z[:4]):
+        assert torch.equal(x, y)

@@ -377,3 +377,17 @@ def test_skipped_block_changes_only_its_rows_weights():
     want = (lf[:, None] * full_o[t, 0] - lbk[:, None] * ob[t, 0]) / (lf - lbk)[:, None]
     np.testing.assert_allclose(o2[t, 0], want, atol=1e-10)
     np.testing.assert_allclose(np.exp(l2[0, t]), lf - lbk, rtol=1e-12)
+
+
+def test_single_row_scoring_equals_full_matrix_row():
+    rng = np.random.default_rng(21)
+    B, s, d, L = 32, 8, 8, 5 * 32 + 9
+    q = rng.standard_normal((L, 4, d))
+    k = rng.standard_normal((L, 2, d))
+    v = rng.standard_normal((L, 2, d)) * 3
+    p = O.Params(block_size=B, stride=s, chunk_size=64, beta=0.3, norm=1.3)
+    full = O.block_scores(q, k, v, [0, L], p)
+    for h in range(4):
+        for i in range(6):
+            row = O.block_score_row(q[:, h:h + 1], k[:, h // 2:h // 2 + 1], v[:, h // 2:h // 2 + 1], i, p)
+            np.testing.assert_allclose(row, full[h, i, :i + 1], rtol=0, atol=1e-12)
