@@ -264,6 +264,7 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.v_scale = qkv->v_scale;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
+  a.q = qkv->q;
   a.out = out;
   a.lse = lse;
   a.status = status;
@@ -271,8 +272,7 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
     BsaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
-      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1) ||
-          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
+      if (!encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
           !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1))
         return STEM_ERR_CUDA;
     }

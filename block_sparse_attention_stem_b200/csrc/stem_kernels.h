@@ -18,8 +18,7 @@ struct ScoreMaps {
 };
 
 struct BsaMaps {
-  CUtensorMap q[kMaxSeqPerLaunch];  // box 128 tokens
-  CUtensorMap k[kMaxSeqPerLaunch];
+  CUtensorMap k[kMaxSeqPerLaunch];  // box 128 tokens
   CUtensorMap v[kMaxSeqPerLaunch];
 };
 
@@ -41,6 +40,7 @@ struct BsaArgs {
   const float* v_scale;
   const int32_t* row_ptr;
   const int32_t* col_idx;
+  const void* q;            // [T, Hq, d] (rows are read straight into TMEM)
   void* out;                // bf16 [T, Hq, d]
   float* lse;               // [Hq][T]
   int* status;
