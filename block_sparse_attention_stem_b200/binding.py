@@ -25,7 +25,7 @@ STATUS_NAMES = {0: "STEM_OK", 1: "STEM_ERR_INVALID_ARG", 2: "STEM_ERR_UNSUPPORTE
                 3: "STEM_ERR_WORKSPACE_TOO_SMALL", 4: "STEM_ERR_MISALIGNED", 5: "STEM_ERR_CUDA",
                 6: "STEM_ERR_TIMEOUT", 7: "STEM_ERR_BAD_BLOCKLIST"}
 STEM_BF16, STEM_FP8_E4M3 = 0, 1
-EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill",
+EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill", "stem_prefill_noalloc",
             "stem_read_device_status", "stem_status_string", "stem_version")
 
 
@@ -69,12 +69,13 @@ def _load() -> ctypes.CDLL:
     lib.stem_select.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_bsa_fwd.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
+    lib.stem_prefill_noalloc.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp]
     lib.stem_read_device_status.argtypes = [vp, vp, P(ctypes.c_int)]
     lib.stem_status_string.argtypes = [ctypes.c_int]
     lib.stem_status_string.restype = ctypes.c_char_p
     lib.stem_version.restype = ctypes.c_int32
     for name in ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill",
-                 "stem_read_device_status"):
+                 "stem_prefill_noalloc", "stem_read_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -221,6 +222,26 @@ def stem_prefill(qkv: QKV, params: StemParams, out=None, lse=None, row_ptr=None,
     _check(LIB.stem_prefill(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(out), _ptr(lse), _ptr(row_ptr),
                             _ptr(col_idx), _ptr(ws), ws.numel(), _stream(stream)), "stem_prefill")
     return out, lse, row_ptr, (None if col_idx is None else col_idx[:pl.nnz]), ws
+
+
+def stem_prefill_noalloc(qkv: QKV, params: StemParams, out=None, lse=None, row_ptr=None, col_idx=None,
+                         stream=None, return_lists=True):
+    """stem_prefill on the library's built-in 32 MiB workspace (for callers that
+    cannot allocate one); the outputs are still the caller's."""
+    pl = stem_plan(qkv, params)
+    dev = qkv.q.device
+    T, hq = qkv.total_tokens, qkv.q.shape[1]
+    if out is None:
+        out = torch.empty(T, hq, 128, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    if return_lists and row_ptr is None:
+        row_ptr = torch.empty(pl.num_rows + 1, dtype=torch.int32, device=dev)
+    if return_lists and col_idx is None:
+        col_idx = torch.empty(max(pl.nnz, 1), dtype=torch.int32, device=dev)
+    _check(LIB.stem_prefill_noalloc(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(out), _ptr(lse),
+                                    _ptr(row_ptr), _ptr(col_idx), _stream(stream)), "stem_prefill_noalloc")
+    return out, lse, row_ptr, (None if col_idx is None else col_idx[:pl.nnz])
 
 
 def stem_read_device_status(ws, stream=None) -> int:

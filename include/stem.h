@@ -186,6 +186,26 @@ STEM_API stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* 
                            int32_t* row_ptr_out, int32_t* col_idx_out,
                            void* ws, size_t ws_bytes, stem_stream_t stream);
 
+/* stem_prefill without a caller workspace, for callers that cannot allocate
+ * device memory (code running where cudaMalloc is not allowed or not wanted:
+ * host callbacks, allocator hooks, plugins whose host owns every device
+ * buffer, fixed memory pools).  The pages have no counterpart: this is a
+ * deployment convenience of this library.
+ *   Uses a built-in 32 MiB device array as the workspace; a problem whose
+ *   plan.ws_prefill_bytes exceeds 32 MiB returns STEM_ERR_WORKSPACE_TOO_SMALL
+ *   before anything is enqueued.  Allocates and frees nothing.
+ *   Every GPU that loads the library keeps the 32 MiB until the process exits.
+ *   All calls on a device share that array and it keeps the last call's
+ *   contents: calls that may overlap on the GPU race; serialise them.
+ *   The first call on each device looks up the array's address (with that
+ *   device current); make it before any stream capture.
+ *   Device-side errors go to the built-in workspace and are not reported here.
+ * Arguments, outputs and host-side errors are those of stem_prefill. */
+STEM_API stem_status_t stem_prefill_noalloc(const stem_qkv_t* qkv, const stem_params_t* params,
+                                            void* out, float* lse,
+                                            int32_t* row_ptr_out, int32_t* col_idx_out,
+                                            stem_stream_t stream);
+
 /* Synchronise `stream` and read the device status word of `ws` into *out.
  * Returns STEM_ERR_CUDA if the copy fails. */
 STEM_API stem_status_t stem_read_device_status(const void* ws, stem_stream_t stream, stem_status_t* out);
