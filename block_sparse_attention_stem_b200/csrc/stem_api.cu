@@ -268,11 +268,13 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.out = out;
   a.lse = lse;
   a.status = status;
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
+  // one CTA per pair of consecutive rows (same query block, neighbouring heads)
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return (hq * si.nb + 1) / 2; })) {
     BsaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
-      if (!encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
+      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1) ||
+          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
           !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1))
         return STEM_ERR_CUDA;
     }

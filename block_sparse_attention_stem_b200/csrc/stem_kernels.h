@@ -18,7 +18,8 @@ struct ScoreMaps {
 };
 
 struct BsaMaps {
-  CUtensorMap k[kMaxSeqPerLaunch];  // box 128 tokens
+  CUtensorMap q[kMaxSeqPerLaunch];  // box 128 tokens
+  CUtensorMap k[kMaxSeqPerLaunch];
   CUtensorMap v[kMaxSeqPerLaunch];
 };
 

@@ -1,0 +1,152 @@
+"""Parity at the full workload sizes, in the launch configuration bench.py times
+(stem_score -> stem_select -> stem_bsa_fwd on one stream).
+
+Every row is checked for what is cheap at any size: budgets and row pointers
+bit-exact against the oracle's closed form; each list strictly ascending,
+ending at the diagonal, containing the sink and window blocks; finite outputs.
+Sampled (query head, query block) rows are checked against the fp64 oracle one
+by one: the block-score row (1e-3 relative), the selected list (exact up to
+near-ties), and the attention output and LSE of the row computed with the
+GPU's list.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import stem_oracle as O
+from block_sparse_attention_stem_b200 import inputs as I
+from gpu_common import TIE_REL, TOL_LSE, TOL_OUT, make_gpu_qkv, out_error
+
+pytestmark = pytest.mark.gpu
+
+b = pytest.importorskip("block_sparse_attention_stem_b200.binding")
+if not torch.cuda.is_available():
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def _run(w):
+    inp = I.make_inputs(w, device="cuda")
+    qkv = make_gpu_qkv(b, inp, w.cu_seqlens())
+    params = b.make_params(**w.params())
+    scores, vbonus, ws = b.stem_score(qkv, params)
+    budgets, row_ptr, col_idx, _ = b.stem_select(qkv, params, scores, ws=ws)
+    out, lse, _ = b.stem_bsa_fwd(qkv, params, row_ptr, col_idx, ws=ws)
+    torch.cuda.synchronize()
+    assert b.stem_read_device_status(ws) == 0
+    return inp, qkv, dict(scores=scores, budgets=budgets, row_ptr=row_ptr, col_idx=col_idx, out=out, lse=lse)
+
+
+def _head_slices(inp, w, s, h):
+    """fp64 single-head arrays of sequence s for query head h (and its KV head)."""
+    cu = w.cu_seqlens()
+    o, e = cu[s], cu[s + 1]
+    G = w.num_q_heads // w.num_kv_heads
+    hk = h // G
+
+    def sl(name, c):
+        x = inp[name][o:e, c:c + 1].contiguous().cpu()
+        if w.dtype == "bf16":
+            return O.dequant(I.raw_bits(x), "bf16")
+        sc = inp[name + "_scale"][c:c + 1].cpu().numpy()
+        return O.dequant(I.raw_bits(x), "fp8", sc)
+
+    return sl("q", h), sl("k", hk), sl("v", hk)
+
+
+def _check_workload(w, samples):
+    inp, qkv, res = _run(w)
+    p = O.Params(**w.params())
+    cu = w.cu_seqlens()
+    seqs, nbtot = O.seq_blocks(cu)
+    hq = w.num_q_heads
+    # --- every row: budgets, row pointers, list structure
+    bud = O.budgets(cu, p)
+    assert np.array_equal(res["budgets"].cpu().numpy(), np.tile(bud, hq))
+    rp = res["row_ptr"].cpu().numpy().astype(np.int64)
+    ci = res["col_idx"].cpu().numpy().astype(np.int64)
+    exp_rp = np.concatenate([[0], np.cumsum(np.tile(bud, hq))])
+    assert np.array_equal(rp, exp_rp)
+    first = np.zeros(len(ci), dtype=bool)
+    first[rp[:-1][rp[:-1] < len(ci)]] = True
+    assert np.all((np.diff(ci) > 0) | first[1:])  # strictly ascending inside each row
+    for (o, L, nb, g0) in seqs:
+        i_of_row = np.arange(nb)
+        last = ci[rp[np.arange(hq)[:, None] * nbtot + g0 + i_of_row[None, :] + 1] - 1]
+        assert np.array_equal(last, np.broadcast_to(i_of_row, last.shape))  # the diagonal ends each row
+    assert torch.isfinite(res["out"].float()).all()
+    assert torch.isfinite(res["lse"]).all()
+    # --- sampled rows against the oracle
+    ties = 0
+    worst = [0.0, 0.0, 0.0]
+    cache = {}
+    for (s, h, i) in samples:
+        o, L, nb, g0 = seqs[s]
+        if (s, h) not in cache:
+            cache = {(s, h): _head_slices(inp, w, s, h)}
+        qh, kh, vh = cache[(s, h)]
+        r = h * nbtot + g0 + i
+        ref_row = O.block_score_row(qh, kh, vh, i, p)
+        gpu_row = res["scores"][h, g0 + i, :i + 1].cpu().numpy().astype(np.float64)
+        err = float(np.max(np.abs(gpu_row - ref_row) / np.maximum(1.0, np.abs(ref_row))))
+        worst[0] = max(worst[0], err)
+        assert err <= 1e-3, (s, h, i, err)
+        G_list = ci[rp[r]:rp[r + 1]]
+        O_list = np.array(O.select_row(ref_row, i, int(bud[g0 + i]), p.sink_blocks, p.window_blocks))
+        if not np.array_equal(G_list, O_list):
+            X = set(G_list.tolist()) - set(O_list.tolist())
+            Y = set(O_list.tolist()) - set(G_list.tolist())
+            assert len(X) == len(Y)
+            for x in X:
+                for y in Y:
+                    assert abs(ref_row[x] - ref_row[y]) < TIE_REL * max(abs(ref_row[x]), abs(ref_row[y]))
+            ties += 1
+        # attention of the row with the GPU's list
+        rp1 = np.zeros(nb + 1, dtype=np.int64)
+        rp1[i + 1:] = len(G_list)
+        ro, rl = O.bsa(qh, kh, vh, [0, L], rp1, G_list, p, rows_subset=[(0, i)])
+        t0, t1 = i * 128, min((i + 1) * 128, L)
+        go = res["out"][o + t0:o + t1, h].float().cpu().numpy().astype(np.float64)
+        gl = res["lse"][h, o + t0:o + t1].cpu().numpy().astype(np.float64)
+        e_o = out_error(go, ro[t0:t1, 0])
+        e_l = float(np.max(np.abs(gl - rl[0, t0:t1])))
+        worst[1] = max(worst[1], e_o)
+        worst[2] = max(worst[2], e_l)
+        assert e_o <= TOL_OUT[w.dtype] and e_l <= TOL_LSE, (s, h, i, e_o, e_l)
+    print(f"{w.name}: rows={len(samples)} near-tie rows={ties} max score err={worst[0]:.2e} "
+          f"max out err={worst[1]:.2e} max lse err={worst[2]:.2e}")
+
+
+def _samples(w, heads, per_seq_blocks):
+    out = []
+    for s, L in enumerate(w.seqlens):
+        nb = math.ceil(L / 128)
+        blocks = sorted({min(nb - 1, x) for x in per_seq_blocks(nb)})
+        for h in heads:
+            for i in blocks:
+                out.append((s, h, i))
+    return out
+
+
+def test_fullsize_qwen32k():
+    w = I.workload("qwen32k")
+    _check_workload(w, _samples(w, (0, 13, 31), lambda nb: (0, 1, 5, nb // 2, nb - 2, nb - 1)))
+
+
+def test_fullsize_long128k_bench_workload():
+    w = I.workload("long128k")
+    _check_workload(w, _samples(w, (0, 17, 31), lambda nb: (0, 3, nb // 3, nb - 1)))
+
+
+@pytest.mark.parametrize("layer", [0, 5])
+def test_fullsize_fp8_varlen_layers(layer):
+    w = I.workload("fp8_varlen", mu=I.fp8_layer_mu(layer), seed=4000 + layer)
+    _check_workload(w, _samples(w, (0, 30), lambda nb: (0, nb // 2, nb - 1)))
+
+
+@pytest.mark.parametrize("rho", [1.0, 0.1])
+def test_fullsize_sweep64k_extremes(rho):
+    w = I.workload("sweep64k", keep_ratio=rho)
+    _check_workload(w, _samples(w, (7,), lambda nb: (2, nb - 1)))
