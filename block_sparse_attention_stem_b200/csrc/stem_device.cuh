@@ -60,24 +60,37 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that lets the hardware suspend the thread until the phase
+// completes (or `hint_ns` elapses), so a waiting warp does not take issue
+// slots from the warps that do the work.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
 // Bounded wait on the phase with the given parity.  Gives up after
 // kWaitLimitNs of wall time (or when another role of the CTA already gave up,
 // signalled through *abort), records STEM_ERR_TIMEOUT and returns false.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s
+constexpr uint32_t kSuspendHintNs = 20000;        // 20 us per suspended try
 
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  uint32_t it = 0;
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((++it & 63u) == 0u) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitLimitNs) {
-        *abort = 1;
-        set_status(status, STEM_ERR_TIMEOUT_CODE);
-        return false;
-      }
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+    if (*abort) return false;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort = 1;
+      set_status(status, STEM_ERR_TIMEOUT_CODE);
+      return false;
     }
   }
 }
@@ -242,6 +255,18 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 }
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Per-warpgroup register budget change (all four warps of a warpgroup execute
+// the same one).  The increases of some warpgroups must be covered by the
+// decreases of others within the CTA's launch allocation, or .inc waits.
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <uint32_t kRegs>
+__device__ __forceinline__ void warpgroup_regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // Named barrier over `nthreads` threads (a multiple of 32).
 __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -263,6 +288,14 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&d);
 }
 
+__device__ __forceinline__ float2 fsub2(float2 a, float2 b) {
+  uint64_t d;
+  asm("sub.f32x2 %0, %1, %2;"
+      : "=l"(d)
+      : "l"(*reinterpret_cast<const uint64_t*>(&a)), "l"(*reinterpret_cast<const uint64_t*>(&b)));
+  return *reinterpret_cast<float2*>(&d);
+}
+
 // Packed fp32 pair arithmetic (sm_100): d = a * b + c on both halves.
 __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
   uint64_t d;
@@ -274,6 +307,25 @@ __device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
 }
 
 // ---------------------------------------------------------------- misc
+// 2^x for a pair, evaluated on the FMA pipes instead of the MUFU unit (Cody-
+// Waite split 2^x = 2^j * 2^f with j = round(x), f in [-1/2, 1/2]; 2^f from a
+// cubic fitted by least squares at 256 Chebyshev nodes of [-1/2, 1/2], max
+// relative error 1.04e-4; 2^j added to the exponent field).  Inputs below
+// -125 return 2^-125; the caller keeps -inf inputs away (masked entries use
+// the MUFU path, which returns exactly 0).
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 magic = make_float2(12582912.f, 12582912.f);  // 1.5 * 2^23: rounds to an integer
+  const float2 t = fadd2(x, magic);                          // j sits in the low mantissa bits
+  const float2 f = fsub2(x, fsub2(t, magic));                // f = x - j in [-1/2, 1/2]
+  float2 p = ffma2(f, make_float2(0.05592203512787819f, 0.05592203512787819f),
+                   make_float2(0.24264007806777954f, 0.24264007806777954f));
+  p = ffma2(p, f, make_float2(0.6931210160255432f, 0.6931210160255432f));
+  p = ffma2(p, f, make_float2(0.9999244809150696f, 0.9999244809150696f));
+  const int jx = __float_as_int(t.x) << 23, jy = __float_as_int(t.y) << 23;  // j << 23
+  return make_float2(__int_as_float(__float_as_int(p.x) + jx), __int_as_float(__float_as_int(p.y) + jy));
+}
 __device__ __forceinline__ float fast_exp2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
@@ -328,3 +380,4 @@ __device__ __forceinline__ int lane_id() { return static_cast<int>(threadIdx.x &
 __device__ __forceinline__ bool elect_one_lane() { return lane_id() == 0; }
 
 }  // namespace stem
+
