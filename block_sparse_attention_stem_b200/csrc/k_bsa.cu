@@ -5,9 +5,9 @@
 // prepared outside it; a skipped block is the same as a block of -inf scores,
 // so the softmax needs no change; fixed 128 x 128 tiles).
 //
-// One CTA owns two CSR rows ("tiles"): consecutive rows in the longest-first
-// order, i.e. the same query block of two neighbouring query heads, whose
-// budgets are equal.  For every listed key block j of a tile (ascending, the
+// One CTA owns two CSR rows ("tiles"): consecutive rows of the KV-head-major,
+// longest-first order, i.e. the same query block of two query heads sharing a
+// KV head, whose budgets are equal.  For every listed key block j of a tile (ascending, the
 // diagonal last):
 //   S = Q K_j^T            tcgen05.mma, Q and K from SMEM, fp32 into the
 //                          tile's TMEM S buffer
@@ -174,11 +174,16 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   Tile tile[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int item = 2 * pair + t;  // rows of a sequence: query blocks descending, heads inner
+    // Rows of a sequence in KV-head-major order: KV head, then query blocks
+    // descending (longest rows first), then the query heads of the group.
+    // CTAs in flight then share one KV head's K/V, which fits in L2.
+    const int item = 2 * pair + t;
     tile[t].valid = item < args.hq * nb;
     const int it = tile[t].valid ? item : 0;
-    tile[t].i = nb - 1 - it / args.hq;
-    tile[t].h = it % args.hq;
+    const int hk_of = it / (G * nb);
+    const int rem = it % (G * nb);
+    tile[t].i = nb - 1 - rem / G;
+    tile[t].h = hk_of * G + rem % G;
     tile[t].hk = tile[t].h / G;
     const size_t r = static_cast<size_t>(tile[t].h) * args.nbtot + batch.g0[seq] + tile[t].i;
     tile[t].beg = tile[t].valid ? args.row_ptr[r] : 0;

@@ -65,9 +65,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
   const int ntile = (nb + s - 1) / s;  // query tiles of 128 groups = s blocks
-  const int I = ntile - 1 - local / args.hq;  // longest rows first
-  const int h = local % args.hq;
-  const int hk = h / (args.hq / args.hkv);
+  // KV-head-major order (KV head, query tiles descending, heads of the group)
+  // so the CTAs in flight share one KV head's keys in L2.
+  const int G = args.hq / args.hkv;
+  const int hk = local / (G * ntile);
+  const int rem = local % (G * ntile);
+  const int I = ntile - 1 - rem / G;  // longest rows first within a KV head
+  const int h = hk * G + rem % G;
   const int halves = kFp8 ? 1 : 2;       // 64-element (bf16) or 128-element (fp8) K chunks per slot
   const int stages_per_tile = s * halves;
   const int rows_per_load = 256 / s;     // TMA box of 256 tokens traversed with stride s
