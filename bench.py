@@ -54,6 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
+    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack"], default="default",
+                    help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack")
+    ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
     return ap.parse_args(argv)
 
 
@@ -479,10 +482,119 @@ def run_reference(args):
     print(json.dumps(res), flush=True)
 
 
+# ---------------------------------------------------------------- extra modes (one GPU)
+def _time_prefill(b, qkv, params, pl, dev, steps, warmup):
+    """Mean CUDA-event time (ms) of the three stages and of the attention
+    stage alone over `steps` runs after `warmup`."""
+    import torch
+    stream = torch.cuda.current_stream()
+    T, hq, hkv = qkv.total_tokens, qkv.q.shape[1], qkv.k.shape[1]
+    scores = torch.empty(hq, pl.nb_total, pl.nb_max, dtype=torch.float32, device=dev)
+    vbonus = torch.empty(hkv, pl.nb_total, dtype=torch.float32, device=dev)
+    budgets = torch.empty(pl.num_rows, dtype=torch.int32, device=dev)
+    row_ptr = torch.empty(pl.num_rows + 1, dtype=torch.int32, device=dev)
+    col_idx = torch.empty(max(pl.nnz, 1), dtype=torch.int32, device=dev)
+    out = torch.empty(T, hq, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    ws = torch.empty(pl.ws_bytes, dtype=torch.uint8, device=dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps + warmup)]
+    for k in range(steps + warmup):
+        ev[k][0].record(stream)
+        b.stem_score(qkv, params, scores, vbonus, ws, stream)
+        ev[k][1].record(stream)
+        b.stem_select(qkv, params, scores, budgets, row_ptr, col_idx, ws, stream)
+        ev[k][2].record(stream)
+        b.stem_bsa_fwd(qkv, params, row_ptr, col_idx, out, lse, ws, stream)
+        ev[k][3].record(stream)
+    torch.cuda.synchronize()
+    status = b.stem_read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(b.stem_status_string(status))
+    tot = sum(e[0].elapsed_time(e[3]) for e in ev[warmup:]) / steps
+    bsa = sum(e[2].elapsed_time(e[3]) for e in ev[warmup:]) / steps
+    return tot, bsa
+
+
+def run_sweep(args):
+    """Latency against kept-block density on the 64K workload with a uniform
+    budget (mu = 1), rho in {1, 0.5, 0.25, 0.2, 0.1}; the pages report the
+    sparse operator's latency as close to linear in density."""
+    import numpy as np
+    import torch
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    w0 = I.workload("sweep64k")
+    inp = I.make_inputs(w0, device="cuda")
+    rows = []
+    sampler = ClockSampler(gpu_device_id(torch))
+    sampler.start()
+    for rho in (1.0, 0.5, 0.25, 0.2, 0.1):
+        w = I.workload("sweep64k", keep_ratio=rho)
+        qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w.cu_seqlens(), cu_seqlens_dev=inp["cu_seqlens"])
+        params = b.make_params(**w.params())
+        pl = b.stem_plan(qkv, params)
+        tot, bsa = _time_prefill(b, qkv, params, pl, dev, args.steps, args.warmup)
+        dens = pl.nnz_per_head / sum(math.ceil(L / 128) * (math.ceil(L / 128) + 1) / 2 for L in w.seqlens)
+        rows.append(dict(rho=rho, density=round(dens, 4), ms=round(tot, 3), bsa_ms=round(bsa, 3),
+                         attn_tflops=round(pl.attn_flops / (bsa * 1e-3) / 1e12, 1)))
+    clocks = sampler.stop()
+    d = np.array([r["density"] for r in rows])
+    fits = {}
+    for key in ("ms", "bsa_ms"):
+        y = np.array([r[key] for r in rows])
+        A = np.vstack([d, np.ones_like(d)]).T
+        (a, c), *_ = np.linalg.lstsq(A, y, rcond=None)
+        dev_rel = np.abs(A @ np.array([a, c]) - y) / y
+        fits[key] = dict(slope_ms_per_density=round(float(a), 3), intercept_ms=round(float(c), 3),
+                         max_rel_deviation=round(float(dev_rel.max()), 4))
+    res = {"metric": "latency vs kept-block density (64K, mu=1)", "unit": "ms", "higher_is_better": False,
+           "points": rows, "linear_fit": fits, "steps": args.steps, "warmup": args.warmup,
+           "config": describe(w0), "clocks": clocks, "dtype": "bf16", "data": "synthetic (seeded, device RNG)"}
+    print(json.dumps(res), flush=True)
+
+
+def run_fp8stack(args):
+    """The fp8 varlen stack: 4 packed sequences {8192, 16384, 40960, 98304},
+    e4m3 inputs with per-head scales, one independently seeded layer per step
+    (mu = 1 for the first 5 layers, 0.7 after), prefill timed per layer."""
+    import torch
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    per_layer = []
+    flops = 0.0
+    sampler = ClockSampler(gpu_device_id(torch))
+    sampler.start()
+    for layer in range(args.layers):
+        w = I.workload("fp8_varlen", mu=I.fp8_layer_mu(layer), seed=4000 + layer)
+        inp = I.make_inputs(w, device="cuda")
+        qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w.cu_seqlens(), q_scale=inp["q_scale"],
+                         k_scale=inp["k_scale"], v_scale=inp["v_scale"], cu_seqlens_dev=inp["cu_seqlens"])
+        params = b.make_params(**w.params())
+        pl = b.stem_plan(qkv, params)
+        tot, bsa = _time_prefill(b, qkv, params, pl, dev, max(1, args.steps // 4), 1)
+        per_layer.append(dict(layer=layer, mu=w.mu, ms=round(tot, 3), bsa_ms=round(bsa, 3)))
+        flops += pl.score_flops + pl.attn_flops
+        del inp, qkv
+    clocks = sampler.stop()
+    total_ms = sum(x["ms"] for x in per_layer)
+    res = {"metric": "fp8 varlen 36-layer stack prefill", "value": round(flops / (total_ms * 1e-3) / 1e12, 2),
+           "unit": UNIT, "total_ms": round(total_ms, 2), "layers": per_layer, "dtype": "e4m3",
+           "config": {"workload": "fp8_varlen: 4 seqs {8192,16384,40960,98304}, 32 Q / 8 KV heads, e4m3, "
+                                  "rho 0.25, mu 1.0 (layers 0-4) / 0.7, sink 4, window 4"},
+           "clocks": clocks, "data": "synthetic (seeded, device RNG)"}
+    print(json.dumps(res), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.impl == "reference":
         run_reference(args)
+    elif args.mode == "sweep":
+        run_sweep(args)
+    elif args.mode == "fp8stack":
+        run_fp8stack(args)
     else:
         run_ours(args)
 

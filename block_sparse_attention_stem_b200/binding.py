@@ -26,7 +26,7 @@ STATUS_NAMES = {0: "STEM_OK", 1: "STEM_ERR_INVALID_ARG", 2: "STEM_ERR_UNSUPPORTE
                 6: "STEM_ERR_TIMEOUT", 7: "STEM_ERR_BAD_BLOCKLIST"}
 STEM_BF16, STEM_FP8_E4M3 = 0, 1
 EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill", "stem_prefill_noalloc",
-            "stem_read_device_status", "stem_status_string", "stem_version")
+            "stem_selftest_wait_timeout", "stem_read_device_status", "stem_status_string", "stem_version")
 
 
 class StemParams(ctypes.Structure):
@@ -70,12 +70,13 @@ def _load() -> ctypes.CDLL:
     lib.stem_bsa_fwd.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill_noalloc.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp]
+    lib.stem_selftest_wait_timeout.argtypes = [vp, vp]
     lib.stem_read_device_status.argtypes = [vp, vp, P(ctypes.c_int)]
     lib.stem_status_string.argtypes = [ctypes.c_int]
     lib.stem_status_string.restype = ctypes.c_char_p
     lib.stem_version.restype = ctypes.c_int32
     for name in ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill",
-                 "stem_prefill_noalloc", "stem_read_device_status"):
+                 "stem_prefill_noalloc", "stem_selftest_wait_timeout", "stem_read_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -242,6 +243,11 @@ def stem_prefill_noalloc(qkv: QKV, params: StemParams, out=None, lse=None, row_p
     _check(LIB.stem_prefill_noalloc(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(out), _ptr(lse),
                                     _ptr(row_ptr), _ptr(col_idx), _stream(stream)), "stem_prefill_noalloc")
     return out, lse, row_ptr, (None if col_idx is None else col_idx[:pl.nnz])
+
+
+def stem_selftest_wait_timeout(ws, stream=None):
+    """Run the bounded-wait self-test; read the result with stem_read_device_status."""
+    _check(LIB.stem_selftest_wait_timeout(_ptr(ws), _stream(stream)), "stem_selftest_wait_timeout")
 
 
 def stem_read_device_status(ws, stream=None) -> int:

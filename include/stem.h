@@ -206,6 +206,14 @@ STEM_API stem_status_t stem_prefill_noalloc(const stem_qkv_t* qkv, const stem_pa
                                             int32_t* row_ptr_out, int32_t* col_idx_out,
                                             stem_stream_t stream);
 
+/* Self-test of the device-side failure detection (no counterpart in the
+ * pages).  Launches one kernel that waits, through the same bounded wait the
+ * pipelines use, on a barrier nothing arrives on; after the 2 s bound it
+ * records STEM_ERR_TIMEOUT in the status word of `ws` (>= 256 bytes) and
+ * returns.  Read the result with stem_read_device_status(); the context stays
+ * usable.  Nothing faults, traps or hangs. */
+STEM_API stem_status_t stem_selftest_wait_timeout(void* ws, stem_stream_t stream);
+
 /* Synchronise `stream` and read the device status word of `ws` into *out.
  * Returns STEM_ERR_CUDA if the copy fails. */
 STEM_API stem_status_t stem_read_device_status(const void* ws, stem_stream_t stream, stem_status_t* out);
