@@ -7,38 +7,41 @@
 //
 // One CTA owns two CSR rows ("tiles"): consecutive rows of the KV-head-major,
 // longest-first order, i.e. the same query block of two query heads sharing a
-// KV head, whose budgets are equal.  For every listed key block j of a tile (ascending, the
-// diagonal last):
-//   S = Q K_j^T            tcgen05.mma, Q and K from SMEM, fp32 into the
-//                          tile's TMEM S buffer
-//   P = exp2(S c - m)      the tile's softmax warpgroup (thread = query row =
-//                          TMEM lane, whole rows, no cross-warp exchange); P is
-//                          written back over S and read from TMEM
-//   O += P V_j             tcgen05.mma, V from SMEM (MN-major), fp32
-//                          accumulator resident in TMEM
-// The two tiles ping-pong: while one softmax warpgroup works, the tensor core
-// runs the other tile's products.  The reference row max m moves (and O is
-// rescaled in TMEM) only when a block raises it past a threshold (2^8 bf16,
-// 2^1 fp8), so P stays bounded and rescales are rare; O and the row sum share
-// that reference, so the result is exact.  Masking happens only on the
-// diagonal block.  A tile's S for block n+1 is issued after its P.V of block
-// n, so the completion of S(n+1) also proves P.V(n) done (one commit tracks
-// every earlier MMA), which is what an O rescale needs.
+// KV head, whose budgets are equal.  Every listed key block j of a tile
+// (ascending, the diagonal last) is processed as two halves of 64 keys,
+// h = 2n and 2n + 1:
+//   S_h = Q K_h^T          tcgen05.mma (M 128, N 64), Q and K from SMEM, fp32
+//                          into S buffer h % 2 of the tile (TMEM)
+//   P_h = exp2(S_h c - m)  the tile's softmax warpgroup (thread = query row =
+//                          TMEM lane); P is written back over S_h
+//   O += P_h V_h           tcgen05.mma with P from TMEM, V from SMEM
+//                          (MN-major); the fp32 accumulator stays in TMEM
+// With two S buffers per tile, S_{h+1} is computed while the softmax of half
+// h runs, so the softmax never waits for the tensor core; the tensor core
+// takes the products of whichever tile is ready (each tile has its own TMA
+// producer and its own MMA issuer).  Both tiles' softmax warps share the
+// SM's exp2 units, which keeps those units busy.
+// The reference row max m moves (and O is rescaled in TMEM) only when a half
+// raises it past a threshold (2^8 bf16, 2^1 fp8), so P stays bounded and
+// rescales are rare; O and the row sum share that reference, so the result is
+// exact.  A rescale first waits for P_{h-1} V_{h-1} (S_h no longer implies it).
+// Masking happens only on the diagonal block.
 //
 // fp8: a single e4m3 P carries three mantissa bits (up to 6% error per weight,
 // which rows with few keys cannot average out), so P*224 is split into
 // hi = e4m3(P*224) and lo = e4m3(remainder); two e4m3 MMAs accumulate hi.V and
 // lo.V into the same O, leaving P about eight significant bits.
 //
-// P is written over S in place, chunk by chunk: chunk ch (keys 32ch..32ch+31)
-// goes to columns 16ch..16ch+15 (bf16 pairs, or 8 columns of hi and 8 of lo
-// for e4m3), which this thread has already read.
+// P is written over S in place: chunk ch (keys 32ch..32ch+31 of the half)
+// goes to columns 16ch..16ch+15 of the S buffer (bf16 pairs, or 8 columns of
+// hi and 8 of lo for e4m3); the whole half is in registers by then.
 //
-// Warp roles (320 threads):
-//   warps 0-3  softmax + epilogue of tile 0 (TMEM lane quarters 0-3)
-//   warps 4-7  softmax + epilogue of tile 1
-//   warp  8    TMA producer: Q of both tiles, then K/V blocks in MMA order
-//   warp  9    TMEM owner and single-thread MMA issuer
+// Warp roles (384 threads):
+//   warps 0-3    softmax + epilogue of tile 0 (TMEM lane quarters 0-3)
+//   warps 4-7    softmax + epilogue of tile 1
+//   warps 8, 9   TMA producer of tile 0, 1: Q, then 64-key halves of K and V
+//                through a per-tile ring, in the order its MMA issuer uses them
+//   warps 10, 11 MMA issuer of tile 0, 1 (warp 10 owns the TMEM allocation)
 // Block lists are staged in shared memory; every wait is bounded.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
@@ -47,16 +50,18 @@ namespace stem {
 
 namespace {
 
-constexpr int kBsaThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr uint32_t kBsaTmemCols = 512;  // tile t: S/P at 256 t, O at 256 t + 128
+constexpr int kBsaThreads = 384;
+constexpr int kProducerWarp = 8;  // + tile
+constexpr int kMmaWarp = 10;      // + tile; warp 10 owns TMEM
+constexpr uint32_t kBsaTmemCols = 512;  // tile t: S buffers at 256 t and 256 t + 64, O at 256 t + 128
+constexpr int kHalf = 64;               // keys per S buffer
 constexpr int kMaxList = 2048;          // list entries per tile staged in SMEM
 
 template <bool kFp8>
 struct BsaCfg {
-  static constexpr int kTileBytes = kFp8 ? 16384 : 32768;  // one 128 x 128 Q, K or V block
-  static constexpr int kSlots = kFp8 ? 8 : 4;              // K/V ring (128 KB)
+  static constexpr int kQBytes = kFp8 ? 16384 : 32768;    // one 128 x 128 Q block
+  static constexpr int kHalfBytes = kFp8 ? 8192 : 16384;  // 64 keys x 128 dims of K or V
+  static constexpr int kSlots = kFp8 ? 8 : 4;             // per-tile ring: 64 KB
   static constexpr float kRescaleLog2 = kFp8 ? 1.f : 8.f;  // max growth before O is rescaled
   static constexpr float kPScale = kFp8 ? 224.f : 1.f;     // P multiplier before rounding (e4m3: 2 * 224 = 448)
 };
@@ -64,15 +69,16 @@ template struct BsaCfg<true>;
 
 template <bool kFp8>
 struct BsaSmem {
-  uint8_t q[2][BsaCfg<kFp8>::kTileBytes];                          // 1024-aligned
-  uint8_t ring[BsaCfg<kFp8>::kSlots][BsaCfg<kFp8>::kTileBytes];
-  uint64_t full[BsaCfg<kFp8>::kSlots];
-  uint64_t empty[BsaCfg<kFp8>::kSlots];
+  uint8_t q[2][BsaCfg<kFp8>::kQBytes];                                   // 1024-aligned
+  uint8_t ring[2][BsaCfg<kFp8>::kSlots][BsaCfg<kFp8>::kHalfBytes];       // per tile
   uint64_t q_full[2];
-  uint64_t s_full[2];  // per tile: S of the current block is in TMEM
-  uint64_t p_full[2];  // per tile: 4 softmax warps stored P (and rescaled O)
-  uint64_t o_done[2];  // per tile: the last P.V is complete
-  uint64_t drain;      // completion of every MMA this CTA issued
+  uint64_t full[2][BsaCfg<kFp8>::kSlots];
+  uint64_t empty[2][BsaCfg<kFp8>::kSlots];
+  uint64_t s_full[2][2];  // per tile and S buffer: S_h complete
+  uint64_t p_full[2][2];  // per tile and S buffer: 4 softmax warps stored P_h (and rescaled O)
+  uint64_t pv_done[2];    // per tile: one phase per completed P_h V_h
+  uint64_t o_done[2];     // per tile: the last P V is complete
+  uint64_t drain[2];      // per tile: every MMA of that tile's issuer complete
   int32_t list[2][kMaxList];
   int nvalid[2];
   int in_smem[2];
@@ -160,7 +166,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     bsa_kernel(const __grid_constant__ BsaMaps maps, const SeqBatch batch, const BsaArgs args) {
   using Cfg = BsaCfg<kFp8>;
   constexpr int kSlots = Cfg::kSlots;
-  constexpr int kHalves = kFp8 ? 1 : 2;  // 64-element (bf16) or 128-element (e4m3) slabs per 128-wide row
+  constexpr int kSlabs = kFp8 ? 1 : 2;  // 128-byte head-dim slabs per row (bf16: dims 0-63 and 64-127)
   extern __shared__ uint8_t smem_raw[];
   BsaSmem<kFp8>& sm =
       *reinterpret_cast<BsaSmem<kFp8>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -190,22 +196,24 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     tile[t].end = tile[t].valid ? args.row_ptr[r + 1] : 0;
   }
 
-  if (warp == kProducerWarp) {
-    stage_list(args.col_idx, tile[0], sm.list[0], &sm.nvalid[0], &sm.in_smem[0], args.status);
+  if (warp == kProducerWarp) stage_list(args.col_idx, tile[0], sm.list[0], &sm.nvalid[0], &sm.in_smem[0], args.status);
+  if (warp == kProducerWarp + 1)
     stage_list(args.col_idx, tile[1], sm.list[1], &sm.nvalid[1], &sm.in_smem[1], args.status);
-  }
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kSlots; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 1);
-    }
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1);
-      mbar_init(&sm.s_full[t], 1);
-      mbar_init(&sm.p_full[t], 4);
+      for (int s = 0; s < kSlots; ++s) {
+        mbar_init(&sm.full[t][s], 1);
+        mbar_init(&sm.empty[t][s], 1);
+      }
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.s_full[t][b], 1);
+        mbar_init(&sm.p_full[t][b], 4);
+      }
+      mbar_init(&sm.pv_done[t], 1);
       mbar_init(&sm.o_done[t], 1);
+      mbar_init(&sm.drain[t], 1);
     }
-    mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -219,127 +227,132 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   const int nv[2] = {sm.nvalid[0], sm.nvalid[1]};
   const bool lsm[2] = {sm.in_smem[0] != 0, sm.in_smem[1] != 0};
-  const int nmax = nv[0] > nv[1] ? nv[0] : nv[1];
   volatile int* abort = &sm.abort;
 
-  if (warp == kProducerWarp) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0 && nmax > 0) {
+  if (warp == kProducerWarp || warp == kProducerWarp + 1) {
+    // ------------------------------------------------------------ producer of tile t
+    const int t = warp - kProducerWarp;
+    const Tile tl = (t == 0) ? tile[0] : tile[1];
+    const int N = (t == 0) ? nv[0] : nv[1];
+    if (lane == 0 && N > 0) {
+      const bool list_in_smem = (t == 0) ? lsm[0] : lsm[1];
       const CUtensorMap* mq = &maps.q[seq];
       const CUtensorMap* mk = &maps.k[seq];
       const CUtensorMap* mv = &maps.v[seq];
       tma_prefetch_desc(mk);
       tma_prefetch_desc(mv);
-#pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        if (nv[t] == 0) continue;
-        mbar_arrive_expect_tx(&sm.q_full[t], Cfg::kTileBytes);
-        for (int hh = 0; hh < kHalves; ++hh)
-          tma_load_3d(sm.q[t] + hh * 16384, mq, &sm.q_full[t], hh * 64, tile[t].h, tile[t].i * kBlock);
-      }
-      ListCursor kc[2] = {ListCursor(tile[0].beg), ListCursor(tile[1].beg)};
-      ListCursor vc[2] = {ListCursor(tile[0].beg), ListCursor(tile[1].beg)};
-      int o = 0;  // ring op counter, in MMA order
-      auto load = [&](const CUtensorMap* m, int t, int j) -> bool {
+      mbar_arrive_expect_tx(&sm.q_full[t], Cfg::kQBytes);
+      for (int hh = 0; hh < kSlabs; ++hh)
+        tma_load_3d(sm.q[t] + hh * 16384, mq, &sm.q_full[t], hh * 64, tl.h, tl.i * kBlock);
+      int o = 0;  // ring ops issued, in the order the MMA issuer consumes them
+      auto load = [&](const CUtensorMap* m, int j, int half) -> bool {
         const int slot = o % kSlots;
-        if (!mbar_wait(&sm.empty[slot], ((o / kSlots) & 1) ^ 1u, abort, args.status)) return false;
-        mbar_arrive_expect_tx(&sm.full[slot], Cfg::kTileBytes);
-        for (int hh = 0; hh < kHalves; ++hh)
-          tma_load_3d(sm.ring[slot] + hh * 16384, m, &sm.full[slot], hh * 64, tile[t].hk, j * kBlock);
+        if (!mbar_wait(&sm.empty[t][slot], ((o / kSlots) & 1) ^ 1u, abort, args.status)) return false;
+        mbar_arrive_expect_tx(&sm.full[t][slot], Cfg::kHalfBytes);
+        for (int hh = 0; hh < kSlabs; ++hh)
+          tma_load_3d(sm.ring[t][slot] + hh * (kHalf * 128), m, &sm.full[t][slot], hh * 64, tl.hk,
+                      j * kBlock + half * kHalf);
         ++o;
         return true;
       };
-      bool ok = true;
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        if (ok && nv[t] > 0) ok = load(mk, t, kc[t].next(sm.list[t], lsm[t], 0, args.col_idx, tile[t].end, tile[t].i));
-      for (int n = 0; n < nmax && ok; ++n) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (ok && n < nv[t])
-            ok = load(mv, t, vc[t].next(sm.list[t], lsm[t], n, args.col_idx, tile[t].end, tile[t].i));
-          if (ok && n + 1 < nv[t])
-            ok = load(mk, t, kc[t].next(sm.list[t], lsm[t], n + 1, args.col_idx, tile[t].end, tile[t].i));
+      // K of halves 0 and 1, then per half h: V_h, K_{h+2}
+      const int H = 2 * N;
+      ListCursor kc(tl.beg), vc(tl.beg);
+      int jk = kc.next(sm.list[t], list_in_smem, 0, args.col_idx, tl.end, tl.i);
+      int jv = 0;
+      bool ok = load(mk, jk, 0) && load(mk, jk, 1);
+      for (int h = 0; h < H && ok; ++h) {
+        if ((h & 1) == 0) jv = vc.next(sm.list[t], list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
+        ok = load(mv, jv, h & 1);
+        if (ok && h + 2 < H) {
+          if ((h & 1) == 0) jk = kc.next(sm.list[t], list_in_smem, (h >> 1) + 1, args.col_idx, tl.end, tl.i);
+          ok = load(mk, jk, h & 1);
         }
+      }
+      // every copy of this producer has landed before the CTA can exit (a
+      // slot holds at most one copy in flight: its next copy waits for the
+      // MMA that consumes this one)
+      mbar_wait_quiesce(&sm.q_full[t], 0, args.status);
+      for (int s = 0; s < kSlots && s < o; ++s) {
+        const int last = s + ((o - 1 - s) / kSlots) * kSlots;  // last op issued into slot s
+        mbar_wait_quiesce(&sm.full[t][s], (last / kSlots) & 1, args.status);
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && nmax > 0) {
-      const uint32_t idesc_s = make_idesc(kFp8 ? 0u : 1u, 0u, 128u, 128u);
+  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
+    // ------------------------------------------------------------ MMA issuer of tile t
+    const int t = warp - kMmaWarp;
+    const int N = (t == 0) ? nv[0] : nv[1];
+    if (lane == 0 && N > 0) {
+      const uint32_t idesc_s = make_idesc(kFp8 ? 0u : 1u, 0u, 128u, static_cast<uint32_t>(kHalf));
       const uint32_t idesc_o = make_idesc(kFp8 ? 0u : 1u, 1u, 128u, 128u);
-      int o = 0;
-      bool ok = true;
-      bool q_ready[2] = {false, false};
-      auto issue_s = [&](int t) -> bool {  // S_t = Q_t K^T from ring op o
-        if (!q_ready[t]) {
-          if (!mbar_wait(&sm.q_full[t], 0, abort, args.status)) return false;
-          q_ready[t] = true;
-        }
+      const uint32_t sq = smem_u32(sm.q[t]);
+      const uint32_t o_tmem = tmem + 256 * t + 128;
+      const int H = 2 * N;
+      int o = 0;  // ring ops consumed
+      auto ring_wait = [&](uint32_t* addr) -> bool {
         const int slot = o % kSlots;
-        if (!mbar_wait(&sm.full[slot], (o / kSlots) & 1, abort, args.status)) return false;
+        if (!mbar_wait(&sm.full[t][slot], (o / kSlots) & 1, abort, args.status)) return false;
         tc_fence_after();
-        const uint32_t sq = smem_u32(sm.q[t]);
-        const uint32_t sk = smem_u32(sm.ring[slot]);
-        const uint32_t d_tmem = tmem + 256 * t;
+        *addr = smem_u32(sm.ring[t][slot]);
+        return true;
+      };
+      auto ring_release = [&]() {  // the slot is reusable once the products just issued complete
+        mma_commit(&sm.empty[t][o % kSlots]);
+        ++o;
+      };
+      auto issue_s = [&](int h) -> bool {  // S_h = Q K_h^T into buffer h % 2
+        uint32_t sk;
+        if (!ring_wait(&sk)) return false;
+        const uint32_t d = tmem + 256 * t + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // 32 head dims per step
-            mma_f8_ss(d_tmem, make_sdesc_sw128(sq + kk * 32, 16, 1024), make_sdesc_sw128(sk + kk * 32, 16, 1024),
-                      idesc_s, kk != 0);
+            mma_f8_ss(d, make_sdesc_sw128(sq + kk * 32, 16, 1024), make_sdesc_sw128(sk + kk * 32, 16, 1024), idesc_s,
+                      kk != 0);
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {  // 16 head dims per step
-            const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-            mma_bf16_ss(d_tmem, make_sdesc_sw128(sq + off, 16, 1024), make_sdesc_sw128(sk + off, 16, 1024), idesc_s,
-                        kk != 0);
-          }
+          for (int kk = 0; kk < 8; ++kk)  // 16 head dims per step
+            mma_bf16_ss(d, make_sdesc_sw128(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                        make_sdesc_sw128(sk + (kk >> 2) * (kHalf * 128) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
         }
-        mma_commit(&sm.s_full[t]);
-        mma_commit(&sm.empty[slot]);
-        ++o;
+        mma_commit(&sm.s_full[t][h & 1]);
+        ring_release();
         return true;
       };
-      auto issue_pv = [&](int t, int n) -> bool {  // O_t += P_t V from ring op o
-        if (!mbar_wait(&sm.p_full[t], n & 1, abort, args.status)) return false;
-        const int slot = o % kSlots;
-        if (!mbar_wait(&sm.full[slot], (o / kSlots) & 1, abort, args.status)) return false;
-        tc_fence_after();
-        const uint32_t sv = smem_u32(sm.ring[slot]);
-        const uint32_t p_tmem = tmem + 256 * t;
-        const uint32_t o_tmem = tmem + 256 * t + 128;
+      auto issue_pv = [&](int h) -> bool {  // O += P_h V_h
+        if (!mbar_wait(&sm.p_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        uint32_t sv;
+        if (!ring_wait(&sv)) return false;
+        const uint32_t p = tmem + 256 * t + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)        // 32 keys per step
+          for (int kk = 0; kk < 2; ++kk)        // 32 keys per step
 #pragma unroll
             for (int part = 0; part < 2; ++part)  // hi at 16 kk, lo at 16 kk + 8
-              mma_f8_ts(o_tmem, p_tmem + kk * 16 + part * 8, make_sdesc_sw128(sv + kk * 4096, 16384, 1024), idesc_o,
-                        (n | part | kk) != 0);
+              mma_f8_ts(o_tmem, p + kk * 16 + part * 8, make_sdesc_sw128(sv + kk * 4096, kHalf * 128, 1024), idesc_o,
+                        (h | part | kk) != 0);
         } else {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)  // 16 keys per step
-            mma_bf16_ts(o_tmem, p_tmem + kk * 8, make_sdesc_sw128(sv + kk * 2048, 16384, 1024), idesc_o,
-                        (n | kk) != 0);
+          for (int kk = 0; kk < 4; ++kk)  // 16 keys per step
+            mma_bf16_ts(o_tmem, p + kk * 8, make_sdesc_sw128(sv + kk * 2048, kHalf * 128, 1024), idesc_o,
+                        (h | kk) != 0);
         }
-        mma_commit(&sm.empty[slot]);
-        if (n == nv[t] - 1) mma_commit(&sm.o_done[t]);
-        ++o;
+        ring_release();
+        mma_commit(&sm.pv_done[t]);
+        if (h == H - 1) mma_commit(&sm.o_done[t]);
         return true;
       };
-#pragma unroll
-      for (int t = 0; t < 2; ++t)
-        if (ok && nv[t] > 0) ok = issue_s(t);
-      for (int n = 0; n < nmax && ok; ++n) {
-#pragma unroll
-        for (int t = 0; t < 2; ++t) {
-          if (ok && n < nv[t]) ok = issue_pv(t, n);
-          if (ok && n + 1 < nv[t]) ok = issue_s(t);
-        }
+      // S_0, S_1, then per half h: P_h V_h and S_{h+2} (into the buffer P_h
+      // V_h just read: one issuer's products run in order)
+      bool ok = mbar_wait(&sm.q_full[t], 0, abort, args.status) && issue_s(0) && issue_s(1);
+      for (int h = 0; h < H && ok; ++h) {
+        ok = issue_pv(h);
+        if (ok && h + 2 < H) ok = issue_s(h + 2);
       }
-      // no MMA may still run when TMEM is released
-      mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0, abort, args.status);
+      // no MMA of this issuer may still run when TMEM is released
+      mma_commit(&sm.drain[t]);
+      mbar_wait_quiesce(&sm.drain[t], 0, args.status);
     }
     __syncwarp();
   } else {
@@ -356,137 +369,130 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
     float c = args.scale_log2;  // sigma * log2(e) (* q_scale * k_scale for fp8)
     if constexpr (kFp8) c *= args.q_scale[tl.h] * args.k_scale[tl.hk];
     const float ninf = -__int_as_float(0x7f800000);
-    const uint32_t s_tmem = tmem + 256 * t + lane_off;
+    const uint32_t s_base = tmem + 256 * t + lane_off;
     const uint32_t o_tmem = tmem + 256 * t + 128 + lane_off;
 
     float m_ref = ninf;  // reference max (scaled log2 domain) shared by O and l
     float l = 0.f;       // row sum of exp2(s c - m_ref)
     bool ok = true;
     ListCursor cur(tl.beg);
-    for (int n = 0; n < N; ++n) {
+    for (int n = 0; n < N && ok; ++n) {
       const int j = cur.next(sm.list[t], list_in_smem, n, args.col_idx, tl.end, tl.i);
       const bool diag = (j == tl.i);
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t], n & 1, abort, args.status))) { ok = false; break; }
-      tc_fence_after();
-      // pass 1: row max of this block (masked on the diagonal); the four
-      // 32-column loads are issued together and waited on once
-      float mx;
-      {
-        uint32_t rr[4][32];
-#pragma unroll
-        for (int ch = 0; ch < 4; ++ch) tmem_ld32(s_tmem + ch * 32, rr[ch]);
+#pragma unroll 1
+      for (int half = 0; half < 2; ++half) {
+        const int h = 2 * n + half;
+        const uint32_t s_tmem = s_base + kHalf * half;
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t][half], n & 1, abort, args.status))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        // the half's 64 scores, loaded once and kept in registers
+        uint32_t rr[2][32];
+        tmem_ld32(s_tmem, rr[0]);
+        tmem_ld32(s_tmem + 32, rr[1]);
         tmem_ld_wait();
         if (diag) {
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch)
+          for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              if (ch * 32 + x > row) rr[ch][x] = 0xff800000u;  // -inf
+              if (half * kHalf + ch * 32 + x > row) rr[ch][x] = 0xff800000u;  // -inf -> p = 0
         }
-        float m8[8];
+        float m4[4];
 #pragma unroll
-        for (int a = 0; a < 8; ++a)
-          m8[a] = fmax3(__uint_as_float(rr[a >> 1][(a & 1) * 16]), __uint_as_float(rr[a >> 1][(a & 1) * 16 + 1]),
+        for (int a = 0; a < 4; ++a)
+          m4[a] = fmax3(__uint_as_float(rr[a >> 1][(a & 1) * 16]), __uint_as_float(rr[a >> 1][(a & 1) * 16 + 1]),
                         __uint_as_float(rr[a >> 1][(a & 1) * 16 + 2]));
 #pragma unroll
         for (int x = 3; x < 15; x += 2)
 #pragma unroll
-          for (int a = 0; a < 8; ++a)
-            m8[a] = fmax3(m8[a], __uint_as_float(rr[a >> 1][(a & 1) * 16 + x]),
+          for (int a = 0; a < 4; ++a)
+            m4[a] = fmax3(m4[a], __uint_as_float(rr[a >> 1][(a & 1) * 16 + x]),
                           __uint_as_float(rr[a >> 1][(a & 1) * 16 + x + 1]));
 #pragma unroll
-        for (int a = 0; a < 8; ++a) m8[a] = fmaxf(m8[a], __uint_as_float(rr[a >> 1][(a & 1) * 16 + 15]));
-        mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
-      }
-      // move the reference only when the max grew past the threshold
-      const float m_cand = mx * c;
-      const bool need = (m_ref == ninf) ? (m_cand != ninf) : (m_cand > m_ref + Cfg::kRescaleLog2);
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? m_cand : m_ref;
-        const float alpha = (m_ref == ninf) ? 0.f : fast_exp2(m_ref - m_new);
-        l *= alpha;
-        if (n >= 1) {  // S(n) complete => P.V(n-1) complete: O may be rescaled now
+        for (int a = 0; a < 4; ++a) m4[a] = fmaxf(m4[a], __uint_as_float(rr[a >> 1][(a & 1) * 16 + 15]));
+        const float m_cand = fmax3(m4[0], m4[1], fmaxf(m4[2], m4[3])) * c;
+        // move the reference only when the max grew past the threshold
+        const bool need = (m_ref == ninf) ? (m_cand != ninf) : (m_cand > m_ref + Cfg::kRescaleLog2);
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? m_cand : m_ref;
+          const float alpha = (m_ref == ninf) ? 0.f : fast_exp2(m_ref - m_new);
+          l *= alpha;
+          if (h >= 1) {
+            // O holds P V up to half h-1: let that product finish first
+            if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t], (h - 1) & 1, abort, args.status))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+#pragma unroll 1
+            for (int ch = 0; ch < 4; ++ch) {
+              uint32_t oo[32];
+              tmem_ld32(o_tmem + ch * 32, oo);
+              tmem_ld_wait();
 #pragma unroll
-          for (int ch = 0; ch < 4; ++ch) {
-            uint32_t rr[32];
-            tmem_ld32(o_tmem + ch * 32, rr);
-            tmem_ld_wait();
+              for (int x = 0; x < 32; ++x) oo[x] = __float_as_uint(__uint_as_float(oo[x]) * alpha);
+              tmem_st32(o_tmem + ch * 32, oo);
+            }
+          }
+          m_ref = m_new;
+        }
+        // p = exp2(s c - m_ref), written over S as the A operand of P V
+        const float m_use = (m_ref == ninf) ? 0.f : m_ref;
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+        float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
 #pragma unroll
-            for (int x = 0; x < 32; ++x) rr[x] = __float_as_uint(__uint_as_float(rr[x]) * alpha);
-            tmem_st32(o_tmem + ch * 32, rr);
+        for (int ch = 0; ch < 2; ++ch) {
+          if constexpr (kFp8) {
+            uint32_t whi[8], wlo[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) {
+              const float2 a = ffma2(make_float2(__uint_as_float(rr[ch][4 * x]), __uint_as_float(rr[ch][4 * x + 1])),
+                                     c2, nm2);
+              const float2 a2 = ffma2(
+                  make_float2(__uint_as_float(rr[ch][4 * x + 2]), __uint_as_float(rr[ch][4 * x + 3])), c2, nm2);
+              const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+              const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+              ps0 = fadd2(ps0, p01);
+              ps1 = fadd2(ps1, p23);
+              const uint32_t x01 = f32x2_to_f16x2(p01.x * Cfg::kPScale, p01.y * Cfg::kPScale);
+              const uint32_t x23 = f32x2_to_f16x2(p23.x * Cfg::kPScale, p23.y * Cfg::kPScale);
+              const uint16_t h01 = f16x2_to_e4m3x2(x01), h23 = f16x2_to_e4m3x2(x23);
+              const uint16_t l01 = f16x2_to_e4m3x2(hsub2_u32(x01, e4m3x2_to_f16x2(h01)));
+              const uint16_t l23 = f16x2_to_e4m3x2(hsub2_u32(x23, e4m3x2_to_f16x2(h23)));
+              whi[x] = static_cast<uint32_t>(h01) | (static_cast<uint32_t>(h23) << 16);
+              wlo[x] = static_cast<uint32_t>(l01) | (static_cast<uint32_t>(l23) << 16);
+            }
+            // 32 keys -> 8 columns of hi at 16 ch and 8 columns of lo at 16 ch + 8
+            tmem_st8(s_tmem + 16 * ch, whi);
+            tmem_st8(s_tmem + 16 * ch + 8, wlo);
+          } else {
+            uint32_t w[16];
+#pragma unroll
+            for (int x = 0; x < 16; x += 2) {
+              const float2 a =
+                  ffma2(make_float2(__uint_as_float(rr[ch][2 * x]), __uint_as_float(rr[ch][2 * x + 1])), c2, nm2);
+              const float2 a2 = ffma2(
+                  make_float2(__uint_as_float(rr[ch][2 * x + 2]), __uint_as_float(rr[ch][2 * x + 3])), c2, nm2);
+              const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
+              const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+              ps0 = fadd2(ps0, p01);
+              ps1 = fadd2(ps1, p23);
+              w[x] = pack_bf16x2(p01.x, p01.y);
+              w[x + 1] = pack_bf16x2(p23.x, p23.y);
+            }
+            // 32 keys -> 16 columns at 16 ch
+            tmem_st16(s_tmem + 16 * ch, w);
           }
         }
-        m_ref = m_new;
+        l += (ps0.x + ps0.y) + (ps1.x + ps1.y);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.p_full[t][half]);
       }
-      // pass 2: p = exp2(s c - m_ref) per 32-column chunk, written over S as the
-      // A operand of P.V (a chunk's P columns never overlap a later chunk's S)
-      const float m_use = (m_ref == ninf) ? 0.f : m_ref;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-      float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
-      uint32_t rr_next[32];
-#pragma unroll
-      for (int ch = 0; ch < 4; ++ch) {
-        // two 32-column loads per wait: chunk ch+1 is fetched with chunk ch
-        uint32_t rr[32];
-        if ((ch & 1) == 0) {
-          tmem_ld32(s_tmem + ch * 32, rr);
-          tmem_ld32(s_tmem + (ch + 1) * 32, rr_next);
-          tmem_ld_wait();
-        } else {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) rr[x] = rr_next[x];
-        }
-        if (diag) {
-#pragma unroll
-          for (int x = 0; x < 32; ++x)
-            if (ch * 32 + x > row) rr[x] = 0xff800000u;  // -inf -> p = 0
-        }
-        if constexpr (kFp8) {
-          uint32_t whi[8], wlo[8];
-#pragma unroll
-          for (int x = 0; x < 8; ++x) {
-            const float2 a = ffma2(make_float2(__uint_as_float(rr[4 * x]), __uint_as_float(rr[4 * x + 1])), c2, nm2);
-            const float2 a2 =
-                ffma2(make_float2(__uint_as_float(rr[4 * x + 2]), __uint_as_float(rr[4 * x + 3])), c2, nm2);
-            const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-            const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-            ps0 = fadd2(ps0, p01);
-            ps1 = fadd2(ps1, p23);
-            const uint32_t x01 = f32x2_to_f16x2(p01.x * Cfg::kPScale, p01.y * Cfg::kPScale);
-            const uint32_t x23 = f32x2_to_f16x2(p23.x * Cfg::kPScale, p23.y * Cfg::kPScale);
-            const uint16_t h01 = f16x2_to_e4m3x2(x01), h23 = f16x2_to_e4m3x2(x23);
-            const uint16_t l01 = f16x2_to_e4m3x2(hsub2_u32(x01, e4m3x2_to_f16x2(h01)));
-            const uint16_t l23 = f16x2_to_e4m3x2(hsub2_u32(x23, e4m3x2_to_f16x2(h23)));
-            whi[x] = static_cast<uint32_t>(h01) | (static_cast<uint32_t>(h23) << 16);
-            wlo[x] = static_cast<uint32_t>(l01) | (static_cast<uint32_t>(l23) << 16);
-          }
-          // 32 keys -> 8 columns of hi at 16 ch and 8 columns of lo at 16 ch + 8,
-          // both inside S columns this thread has already read
-          tmem_st8(s_tmem + 16 * ch, whi);
-          tmem_st8(s_tmem + 16 * ch + 8, wlo);
-        } else {
-          uint32_t w[16];
-#pragma unroll
-          for (int x = 0; x < 16; x += 2) {
-            const float2 a = ffma2(make_float2(__uint_as_float(rr[2 * x]), __uint_as_float(rr[2 * x + 1])), c2, nm2);
-            const float2 a2 =
-                ffma2(make_float2(__uint_as_float(rr[2 * x + 2]), __uint_as_float(rr[2 * x + 3])), c2, nm2);
-            const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-            const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-            ps0 = fadd2(ps0, p01);
-            ps1 = fadd2(ps1, p23);
-            w[x] = pack_bf16x2(p01.x, p01.y);
-            w[x + 1] = pack_bf16x2(p23.x, p23.y);
-          }
-          // 32 keys -> 16 columns at 16 ch
-          tmem_st16(s_tmem + 16 * ch, w);
-        }
-      }
-      l += (ps0.x + ps0.y) + (ps1.x + ps1.y);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.p_full[t]);
     }
 
     // epilogue: normalise O and store this row (the TMEM reads are warp-wide;

@@ -273,9 +273,11 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
     BsaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
+      // Q in 128-token boxes; K and V in 64-token boxes (the attention
+      // kernel moves half a key block per copy)
       if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1) ||
-          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1) ||
-          !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock, 1))
+          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1) ||
+          !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1))
         return STEM_ERR_CUDA;
     }
     stem_status_t st = cuda_status(launch_bsa(maps, b, a, fp8, stream));

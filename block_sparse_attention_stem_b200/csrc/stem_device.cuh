@@ -95,6 +95,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
   }
 }
 
+// Bounded wait used on the way out (also after an abort): waits for this
+// role's own asynchronous work (copies or products in flight) to finish, so
+// that no copy lands in, and no product writes, memory the CTA is releasing.
+// Ignores *abort; gives up only after kWaitLimitNs, recording STEM_ERR_TIMEOUT.
+__device__ __forceinline__ bool mbar_wait_quiesce(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  while (true) {
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+    if (globaltimer_ns() - t0 > kWaitLimitNs) {
+      set_status(status, STEM_ERR_TIMEOUT_CODE);
+      return false;
+    }
+  }
+}
+
 // ---------------------------------------------------------------- fences
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
