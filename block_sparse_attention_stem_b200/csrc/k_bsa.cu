@@ -36,12 +36,17 @@
 // goes to columns 16ch..16ch+15 of the S buffer (bf16 pairs, or 8 columns of
 // hi and 8 of lo for e4m3); the whole half is in registers by then.
 //
-// Warp roles (384 threads):
+// Warp roles (448 threads):
 //   warps 0-3    softmax + epilogue of tile 0 (TMEM lane quarters 0-3)
 //   warps 4-7    softmax + epilogue of tile 1
-//   warps 8, 9   TMA producer of tile 0, 1: Q, then 64-key halves of K and V
-//                through a per-tile ring, in the order its MMA issuer uses them
-//   warps 10, 11 MMA issuer of tile 0, 1 (warp 10 owns the TMEM allocation)
+//   warps 8-11   TMA producers: tile 0 Q and K, tile 0 V, tile 1 Q and K,
+//                tile 1 V (64-key halves)
+//   warps 12, 13 MMA issuer of tile 0, 1 (warp 12 owns the TMEM allocation)
+// Each tile has two K slots and two V slots (half h uses slot h % 2).  The
+// completion of S_h frees K slot h % 2 and that of P_h V_h frees V slot h % 2,
+// so a product needs one commit.  Tile 1 starts once tile 0 has stored its
+// first P, which staggers the two softmax warpgroups: while one computes
+// exponentials the other is in its row-max and bookkeeping phase.
 // Block lists are staged in shared memory; every wait is bounded.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
@@ -50,18 +55,23 @@ namespace stem {
 
 namespace {
 
-constexpr int kBsaThreads = 384;
-constexpr int kProducerWarp = 8;  // + tile
-constexpr int kMmaWarp = 10;      // + tile; warp 10 owns TMEM
+constexpr int kBsaThreads = 448;
+constexpr int kProducerWarp = 8;  // + 2 tile + (0: Q and K, 1: V)
+constexpr int kMmaWarp = 12;      // + tile; warp 12 owns TMEM
 constexpr uint32_t kBsaTmemCols = 512;  // tile t: S buffers at 256 t and 256 t + 64, O at 256 t + 128
 constexpr int kHalf = 64;               // keys per S buffer
 constexpr int kMaxList = 2048;          // list entries per tile staged in SMEM
+// Pairs of keys (bit k: keys 2k, 2k+1 of a 32-key chunk) whose exp2 runs on
+// the FMA pipes (exp2_poly2) instead of the MUFU unit, off the diagonal block.
+#ifndef STEM_BSA_POLY_MASK
+#define STEM_BSA_POLY_MASK 0x2222u
+#endif
+constexpr uint32_t kPolyMask = STEM_BSA_POLY_MASK;
 
 template <bool kFp8>
 struct BsaCfg {
   static constexpr int kQBytes = kFp8 ? 16384 : 32768;    // one 128 x 128 Q block
   static constexpr int kHalfBytes = kFp8 ? 8192 : 16384;  // 64 keys x 128 dims of K or V
-  static constexpr int kSlots = kFp8 ? 8 : 4;             // per-tile ring: 64 KB
   static constexpr float kRescaleLog2 = kFp8 ? 1.f : 8.f;  // max growth before O is rescaled
   static constexpr float kPScale = kFp8 ? 224.f : 1.f;     // P multiplier before rounding (e4m3: 2 * 224 = 448)
 };
@@ -70,15 +80,17 @@ template struct BsaCfg<true>;
 template <bool kFp8>
 struct BsaSmem {
   uint8_t q[2][BsaCfg<kFp8>::kQBytes];                                   // 1024-aligned
-  uint8_t ring[2][BsaCfg<kFp8>::kSlots][BsaCfg<kFp8>::kHalfBytes];       // per tile
+  uint8_t k[2][2][BsaCfg<kFp8>::kHalfBytes];  // per tile, per slot
+  uint8_t v[2][2][BsaCfg<kFp8>::kHalfBytes];
   uint64_t q_full[2];
-  uint64_t full[2][BsaCfg<kFp8>::kSlots];
-  uint64_t empty[2][BsaCfg<kFp8>::kSlots];
-  uint64_t s_full[2][2];  // per tile and S buffer: S_h complete
+  uint64_t k_full[2][2];  // per tile and slot: K_h landed
+  uint64_t v_full[2][2];  // per tile and slot: V_h landed
+  uint64_t s_full[2][2];  // per tile and S buffer: S_h complete (K slot free again)
+  uint64_t v_free[2][2];  // per tile and slot: P_h V_h complete (V slot free again)
   uint64_t p_full[2][2];  // per tile and S buffer: 4 softmax warps stored P_h (and rescaled O)
-  uint64_t pv_done[2];    // per tile: one phase per completed P_h V_h
   uint64_t o_done[2];     // per tile: the last P V is complete
   uint64_t drain[2];      // per tile: every MMA of that tile's issuer complete
+  uint64_t stagger;       // tile 0 stored its first P
   int32_t list[2][kMaxList];
   int nvalid[2];
   int in_smem[2];
@@ -159,13 +171,31 @@ __device__ void stage_list(const int32_t* __restrict__ col, const Tile& t, int32
   }
 }
 
+// p = exp2(s c - m) for one 32-key chunk of a row: packed scale-and-shift,
+// exp2 (MUFU, or for the pairs in kPoly the FMA-pipe polynomial), packed row
+// sums and bf16 packing.  w[k] holds keys 2k (low half) and 2k + 1.
+template <uint32_t kPoly>
+__device__ __forceinline__ void exp_chunk_bf16(const uint32_t* rr, float2 c2, float2 nm2, float2& ps0, float2& ps1,
+                                               uint32_t* w) {
+#pragma unroll
+  for (int x = 0; x < 16; x += 2) {
+    const float2 a = ffma2(make_float2(__uint_as_float(rr[2 * x]), __uint_as_float(rr[2 * x + 1])), c2, nm2);
+    const float2 a2 = ffma2(make_float2(__uint_as_float(rr[2 * x + 2]), __uint_as_float(rr[2 * x + 3])), c2, nm2);
+    const float2 p01 = ((kPoly >> x) & 1u) ? exp2_poly2(a) : make_float2(fast_exp2(a.x), fast_exp2(a.y));
+    const float2 p23 = ((kPoly >> (x + 1)) & 1u) ? exp2_poly2(a2) : make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
+    ps0 = fadd2(ps0, p01);
+    ps1 = fadd2(ps1, p23);
+    w[x] = pack_bf16x2(p01.x, p01.y);
+    w[x + 1] = pack_bf16x2(p23.x, p23.y);
+  }
+}
+
 }  // namespace
 
 template <bool kFp8>
 __global__ void __launch_bounds__(kBsaThreads, 1)
     bsa_kernel(const __grid_constant__ BsaMaps maps, const SeqBatch batch, const BsaArgs args) {
   using Cfg = BsaCfg<kFp8>;
-  constexpr int kSlots = Cfg::kSlots;
   constexpr int kSlabs = kFp8 ? 1 : 2;  // 128-byte head-dim slabs per row (bf16: dims 0-63 and 64-127)
   extern __shared__ uint8_t smem_raw[];
   BsaSmem<kFp8>& sm =
@@ -197,23 +227,22 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   }
 
   if (warp == kProducerWarp) stage_list(args.col_idx, tile[0], sm.list[0], &sm.nvalid[0], &sm.in_smem[0], args.status);
-  if (warp == kProducerWarp + 1)
+  if (warp == kProducerWarp + 2)
     stage_list(args.col_idx, tile[1], sm.list[1], &sm.nvalid[1], &sm.in_smem[1], args.status);
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
       mbar_init(&sm.q_full[t], 1);
-      for (int s = 0; s < kSlots; ++s) {
-        mbar_init(&sm.full[t][s], 1);
-        mbar_init(&sm.empty[t][s], 1);
-      }
       for (int b = 0; b < 2; ++b) {
+        mbar_init(&sm.k_full[t][b], 1);
+        mbar_init(&sm.v_full[t][b], 1);
         mbar_init(&sm.s_full[t][b], 1);
+        mbar_init(&sm.v_free[t][b], 1);
         mbar_init(&sm.p_full[t][b], 4);
       }
-      mbar_init(&sm.pv_done[t], 1);
       mbar_init(&sm.o_done[t], 1);
       mbar_init(&sm.drain[t], 1);
     }
+    mbar_init(&sm.stagger, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -229,53 +258,49 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   const bool lsm[2] = {sm.in_smem[0] != 0, sm.in_smem[1] != 0};
   volatile int* abort = &sm.abort;
 
-  if (warp == kProducerWarp || warp == kProducerWarp + 1) {
-    // ------------------------------------------------------------ producer of tile t
-    const int t = warp - kProducerWarp;
+  if (warp >= kProducerWarp && warp < kProducerWarp + 4) {
+    // ------------------------------------------------------------ producers
+    // warp 8 + 2 t + kind: kind 0 loads Q and the K halves of tile t, kind 1
+    // the V halves (one issuing thread moves only about 26 B per cycle, so
+    // K and V get a thread each)
+    const int t = (warp - kProducerWarp) >> 1;
+    const bool is_v = ((warp - kProducerWarp) & 1) != 0;
     const Tile tl = (t == 0) ? tile[0] : tile[1];
     const int N = (t == 0) ? nv[0] : nv[1];
     if (lane == 0 && N > 0) {
       const bool list_in_smem = (t == 0) ? lsm[0] : lsm[1];
-      const CUtensorMap* mq = &maps.q[seq];
-      const CUtensorMap* mk = &maps.k[seq];
-      const CUtensorMap* mv = &maps.v[seq];
-      tma_prefetch_desc(mk);
-      tma_prefetch_desc(mv);
-      mbar_arrive_expect_tx(&sm.q_full[t], Cfg::kQBytes);
-      for (int hh = 0; hh < kSlabs; ++hh)
-        tma_load_3d(sm.q[t] + hh * 16384, mq, &sm.q_full[t], hh * 64, tl.h, tl.i * kBlock);
-      int o = 0;  // ring ops issued, in the order the MMA issuer consumes them
-      auto load = [&](const CUtensorMap* m, int j, int half) -> bool {
-        const int slot = o % kSlots;
-        if (!mbar_wait(&sm.empty[t][slot], ((o / kSlots) & 1) ^ 1u, abort, args.status)) return false;
-        mbar_arrive_expect_tx(&sm.full[t][slot], Cfg::kHalfBytes);
+      const CUtensorMap* m = is_v ? &maps.v[seq] : &maps.k[seq];
+      tma_prefetch_desc(m);
+      if (!is_v) {
+        mbar_arrive_expect_tx(&sm.q_full[t], Cfg::kQBytes);
         for (int hh = 0; hh < kSlabs; ++hh)
-          tma_load_3d(sm.ring[t][slot] + hh * (kHalf * 128), m, &sm.full[t][slot], hh * 64, tl.hk,
-                      j * kBlock + half * kHalf);
-        ++o;
-        return true;
-      };
-      // K of halves 0 and 1, then per half h: V_h, K_{h+2}
+          tma_load_3d(sm.q[t] + hh * 16384, &maps.q[seq], &sm.q_full[t], hh * 64, tl.h, tl.i * kBlock);
+      }
+      // Half h goes to slot h % 2.  K_{h+2} may overwrite K_h once S_h is
+      // complete, V_{h+2} may overwrite V_h once P_h V_h is.
       const int H = 2 * N;
-      ListCursor kc(tl.beg), vc(tl.beg);
-      int jk = kc.next(sm.list[t], list_in_smem, 0, args.col_idx, tl.end, tl.i);
-      int jv = 0;
-      bool ok = load(mk, jk, 0) && load(mk, jk, 1);
-      for (int h = 0; h < H && ok; ++h) {
-        if ((h & 1) == 0) jv = vc.next(sm.list[t], list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
-        ok = load(mv, jv, h & 1);
-        if (ok && h + 2 < H) {
-          if ((h & 1) == 0) jk = kc.next(sm.list[t], list_in_smem, (h >> 1) + 1, args.col_idx, tl.end, tl.i);
-          ok = load(mk, jk, h & 1);
+      ListCursor cur(tl.beg);
+      int j = 0, issued = 0;
+      for (int h = 0; h < H; ++h) {
+        if (h >= 2) {
+          uint64_t* freed = is_v ? &sm.v_free[t][h & 1] : &sm.s_full[t][h & 1];
+          if (!mbar_wait(freed, ((h - 2) >> 1) & 1, abort, args.status)) break;
         }
+        if ((h & 1) == 0) j = cur.next(sm.list[t], list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
+        uint8_t* dst = is_v ? sm.v[t][h & 1] : sm.k[t][h & 1];
+        uint64_t* bar = is_v ? &sm.v_full[t][h & 1] : &sm.k_full[t][h & 1];
+        mbar_arrive_expect_tx(bar, Cfg::kHalfBytes);
+        for (int hh = 0; hh < kSlabs; ++hh)
+          tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, j * kBlock + (h & 1) * kHalf);
+        ++issued;
       }
       // every copy of this producer has landed before the CTA can exit (a
-      // slot holds at most one copy in flight: its next copy waits for the
-      // MMA that consumes this one)
-      mbar_wait_quiesce(&sm.q_full[t], 0, args.status);
-      for (int s = 0; s < kSlots && s < o; ++s) {
-        const int last = s + ((o - 1 - s) / kSlots) * kSlots;  // last op issued into slot s
-        mbar_wait_quiesce(&sm.full[t][s], (last / kSlots) & 1, args.status);
+      // slot holds at most one copy in flight: the next copy into it waits
+      // for the product that consumes this one)
+      if (!is_v) mbar_wait_quiesce(&sm.q_full[t], 0, args.status);
+      for (int x = 0; x < 2 && x < issued; ++x) {
+        const int last = issued - 1 - ((issued - 1 - x) & 1);  // last half issued into slot x
+        mbar_wait_quiesce(is_v ? &sm.v_full[t][x] : &sm.k_full[t][x], (last >> 1) & 1, args.status);
       }
     }
     __syncwarp();
@@ -289,21 +314,10 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       const uint32_t sq = smem_u32(sm.q[t]);
       const uint32_t o_tmem = tmem + 256 * t + 128;
       const int H = 2 * N;
-      int o = 0;  // ring ops consumed
-      auto ring_wait = [&](uint32_t* addr) -> bool {
-        const int slot = o % kSlots;
-        if (!mbar_wait(&sm.full[t][slot], (o / kSlots) & 1, abort, args.status)) return false;
-        tc_fence_after();
-        *addr = smem_u32(sm.ring[t][slot]);
-        return true;
-      };
-      auto ring_release = [&]() {  // the slot is reusable once the products just issued complete
-        mma_commit(&sm.empty[t][o % kSlots]);
-        ++o;
-      };
       auto issue_s = [&](int h) -> bool {  // S_h = Q K_h^T into buffer h % 2
-        uint32_t sk;
-        if (!ring_wait(&sk)) return false;
+        if (!mbar_wait(&sm.k_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        tc_fence_after();
+        const uint32_t sk = smem_u32(sm.k[t][h & 1]);
         const uint32_t d = tmem + 256 * t + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
@@ -317,13 +331,13 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
                         make_sdesc_sw128(sk + (kk >> 2) * (kHalf * 128) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
         }
         mma_commit(&sm.s_full[t][h & 1]);
-        ring_release();
         return true;
       };
       auto issue_pv = [&](int h) -> bool {  // O += P_h V_h
         if (!mbar_wait(&sm.p_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
-        uint32_t sv;
-        if (!ring_wait(&sv)) return false;
+        if (!mbar_wait(&sm.v_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        tc_fence_after();
+        const uint32_t sv = smem_u32(sm.v[t][h & 1]);
         const uint32_t p = tmem + 256 * t + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
@@ -338,14 +352,15 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
             mma_bf16_ts(o_tmem, p + kk * 8, make_sdesc_sw128(sv + kk * 2048, kHalf * 128, 1024), idesc_o,
                         (h | kk) != 0);
         }
-        ring_release();
-        mma_commit(&sm.pv_done[t]);
+        mma_commit(&sm.v_free[t][h & 1]);
         if (h == H - 1) mma_commit(&sm.o_done[t]);
         return true;
       };
+      // tile 1 starts once tile 0 stored its first P (see the header)
+      bool ok = !(t == 1 && nv[0] > 0) || mbar_wait(&sm.stagger, 0, abort, args.status);
       // S_0, S_1, then per half h: P_h V_h and S_{h+2} (into the buffer P_h
       // V_h just read: one issuer's products run in order)
-      bool ok = mbar_wait(&sm.q_full[t], 0, abort, args.status) && issue_s(0) && issue_s(1);
+      ok = ok && mbar_wait(&sm.q_full[t], 0, abort, args.status) && issue_s(0) && issue_s(1);
       for (int h = 0; h < H && ok; ++h) {
         ok = issue_pv(h);
         if (ok && h + 2 < H) ok = issue_s(h + 2);
@@ -422,7 +437,8 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           l *= alpha;
           if (h >= 1) {
             // O holds P V up to half h-1: let that product finish first
-            if (!__all_sync(0xffffffffu, mbar_wait(&sm.pv_done[t], (h - 1) & 1, abort, args.status))) {
+            if (!__all_sync(0xffffffffu,
+                            mbar_wait(&sm.v_free[t][(h - 1) & 1], ((h - 1) >> 1) & 1, abort, args.status))) {
               ok = false;
               break;
             }
@@ -470,18 +486,10 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
             tmem_st8(s_tmem + 16 * ch + 8, wlo);
           } else {
             uint32_t w[16];
-#pragma unroll
-            for (int x = 0; x < 16; x += 2) {
-              const float2 a =
-                  ffma2(make_float2(__uint_as_float(rr[ch][2 * x]), __uint_as_float(rr[ch][2 * x + 1])), c2, nm2);
-              const float2 a2 = ffma2(
-                  make_float2(__uint_as_float(rr[ch][2 * x + 2]), __uint_as_float(rr[ch][2 * x + 3])), c2, nm2);
-              const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-              const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-              ps0 = fadd2(ps0, p01);
-              ps1 = fadd2(ps1, p23);
-              w[x] = pack_bf16x2(p01.x, p01.y);
-              w[x + 1] = pack_bf16x2(p23.x, p23.y);
+            if (diag) {
+              exp_chunk_bf16<0u>(rr[ch], c2, nm2, ps0, ps1, w);  // masked keys need an exact 0
+            } else {
+              exp_chunk_bf16<kPolyMask>(rr[ch], c2, nm2, ps0, ps1, w);
             }
             // 32 keys -> 16 columns at 16 ch
             tmem_st16(s_tmem + 16 * ch, w);
@@ -492,6 +500,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.p_full[t][half]);
+        if (t == 0 && h == 0 && warp == 0 && lane == 0) mbar_arrive(&sm.stagger);
       }
     }
 
