@@ -176,13 +176,16 @@ def load_peaks():
         return FALLBACK_PEAKS, "fallback"
 
 
-def bsa_traffic_per_launch():
+def bsa_traffic_per_launch(workload: str):
     """dram bytes per launch of the attention kernel from the committed ncu
-    summary, valid only while the kernel source is the one that was profiled."""
+    summary, valid only for the workload it was captured on and while the
+    kernel source is the one that was profiled."""
     try:
         rec = dict(line.split(None, 1) for line in open(TRAFFIC_FILE) if line.strip() and not line.startswith("#"))
         src = open(os.path.join(ROOT, "block_sparse_attention_stem_b200", "csrc", "k_bsa.cu"), "rb").read()
         if rec.get("source_sha256", "").strip() != hashlib.sha256(src).hexdigest():
+            return None
+        if rec.get("workload", "").strip() != workload:
             return None
         return float(rec["bytes_per_launch_full_workload"])
     except (OSError, ValueError, KeyError):
@@ -409,7 +412,7 @@ def run_ours(args):
     if w.dtype == "fp8":
         peak *= 2.0  # nominal fp8 : bf16 dense ratio
     achieved = pl.attn_flops / (bsa_ms * 1e-3) / 1e12
-    traffic = bsa_traffic_per_launch() if w.dtype == "bf16" else None
+    traffic = bsa_traffic_per_launch(w.name)
     roofline = {"bound": "tensor", "kernel": "bsa_kernel", "achieved": round(achieved, 2), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if w.dtype == "fp8"
