@@ -64,7 +64,7 @@ constexpr int kMaxList = 2048;          // list entries per tile staged in SMEM
 // Pairs of keys (bit k: keys 2k, 2k+1 of a 32-key chunk) whose exp2 runs on
 // the FMA pipes (exp2_poly2) instead of the MUFU unit, off the diagonal block.
 #ifndef STEM_BSA_POLY_MASK
-#define STEM_BSA_POLY_MASK 0x2222u
+#define STEM_BSA_POLY_MASK 0x0u
 #endif
 constexpr uint32_t kPolyMask = STEM_BSA_POLY_MASK;
 
