@@ -9,20 +9,24 @@
 //
 // D is a plain GEMM with reduction length s*d: query group a contributes the
 // s token rows a s + u (slot u), key group b the rows b s + s-1-u.  Each CTA
-// owns one (sequence, query head, 128-group query tile I) and walks the
-// 256-group key tiles J that reach its causal range.  Slot tiles are fetched
-// by TMA with a token traversal stride of s (one tensor map per sequence, so
-// rows past the sequence end arrive as zeros), staged 128-B swizzled, and fed
-// to tcgen05.mma (M = 128, N = 256, fp32 in TMEM, two accumulators so the
-// epilogue of tile J overlaps the MMAs of J+1).  N = 256 makes every A read
-// from shared memory serve twice as many products as N = 128, which is what
-// bounds this GEMM (each operand byte is read from SMEM once per MMA).
-// The epilogue warps read their TMEM lane quarter, max-pool 16 columns in
-// registers and 16 rows with warp shuffles, scale, add the bonus and write one
-// fp32 score per (query block, key block).
+// owns one (sequence, pair of query heads of one KV group, 128-group query
+// tile I) and walks the 256-group key tiles J that reach its causal range.
+// Slot tiles are fetched by TMA with a token traversal stride of s (one tensor
+// map per sequence, so rows past the sequence end arrive as zeros), staged
+// 128-B swizzled, and fed to tcgen05.mma (M = 128, N = 256, fp32 in TMEM, one
+// 256-column accumulator per head).  The two heads share every staged key
+// tile: a 64 KB stage (two 16 KB query slabs, one 32 KB key slab) feeds 1024
+// tensor cycles, where a single head's 48 KB stage fed 512.  The bytes moved
+// from L2 into shared memory per product are what bound this GEMM, so sharing
+// the key slab is what pays.  The epilogue warps (one warpgroup per head) read
+// their TMEM lane quarter, max-pool 16 columns in registers and 16 rows with
+// warp shuffles, scale, add the bonus and write one fp32 score per (query
+// block, key block); the next tile's products on a head wait only for that
+// head's epilogue.
 //
-// Warp roles (192 threads): warp 0 TMA producer, warp 1 TMEM owner + MMA
-// issuer, warps 2-5 epilogue (TMEM lane quarters 2, 3, 0, 1).
+// Warp roles (320 threads): warps 0-3 epilogue of the first head, warps 4-7 of
+// the second (TMEM lane quarter = warp % 4), warp 8 TMA producer, warp 9 TMEM
+// owner + MMA issuer.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
 
@@ -30,22 +34,24 @@ namespace stem {
 
 namespace {
 
-constexpr int kScoreThreads = 192;
+constexpr int kScoreThreads = 320;
+constexpr int kProducerWarp = 8;
+constexpr int kMmaWarp = 9;
 constexpr int kTileM = 128;            // query groups per tile (MMA M)
 constexpr int kTileN = 256;            // key groups per tile (MMA N)
-constexpr int kBytesA = kTileM * 128;  // one 128-B row per group and K-chunk
+constexpr int kBytesA = kTileM * 128;  // one 128-B row per group and K-chunk, per head
 constexpr int kBytesB = kTileN * 128;
-constexpr int kStageBytes = kBytesA + kBytesB;  // 48 KB
-constexpr int kScoreStages = 4;
-constexpr uint32_t kScoreTmemCols = 512;  // two 256-column accumulators
+constexpr int kStageBytes = 2 * kBytesA + kBytesB;  // 64 KB: A of both heads, then B
+constexpr int kScoreStages = 3;
+constexpr uint32_t kScoreTmemCols = 512;  // head e: 256-column accumulator at 256 e
 
 struct ScoreSmem {
   uint8_t stage[kScoreStages][kStageBytes];  // 1024-aligned (swizzle atoms)
   uint64_t full[kScoreStages];
   uint64_t empty[kScoreStages];
-  uint64_t acc_full[2];
-  uint64_t acc_empty[2];
-  uint64_t drain;  // completion of every MMA this CTA issued
+  uint64_t acc_full;      // the products of tile J are complete (both heads)
+  uint64_t acc_empty[2];  // per head: its epilogue read tile J
+  uint64_t drain;         // completion of every MMA this CTA issued
   uint32_t tmem_base;
   int abort;
 };
@@ -65,13 +71,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
   const int ntile = (nb + s - 1) / s;  // query tiles of 128 groups = s blocks
-  // KV-head-major order (KV head, query tiles descending, heads of the group)
-  // so the CTAs in flight share one KV head's keys in L2.
+  // KV-head-major order (KV head, query tiles descending, head pairs of the
+  // group) so the CTAs in flight share one KV head's keys in L2.
   const int G = args.hq / args.hkv;
-  const int hk = local / (G * ntile);
-  const int rem = local % (G * ntile);
-  const int I = ntile - 1 - rem / G;  // longest rows first within a KV head
-  const int h = hk * G + rem % G;
+  const int npair = (G + 1) / 2;
+  const int hk = local / (npair * ntile);
+  const int rem = local % (npair * ntile);
+  const int I = ntile - 1 - rem / npair;  // longest rows first within a KV head
+  const int h0 = hk * G + 2 * (rem % npair);
+  const bool has1 = 2 * (rem % npair) + 1 < G;  // an odd group leaves the last pair one head
   const int halves = kFp8 ? 1 : 2;       // 64-element (bf16) or 128-element (fp8) K chunks per slot
   const int stages_per_tile = s * halves;
   const int rows_per_load = 256 / s;     // TMA box of 256 tokens traversed with stride s
@@ -85,15 +93,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       mbar_init(&sm.full[i], 1);
       mbar_init(&sm.empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.acc_full[i], 1);
-      mbar_init(&sm.acc_empty[i], 4);
-    }
+    mbar_init(&sm.acc_full, 1);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.acc_empty[i], 4);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&sm.tmem_base, kScoreTmemCols);
     tmem_relinquish();
   }
@@ -103,7 +109,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const uint32_t tmem = sm.tmem_base;
   volatile int* abort = &sm.abort;
 
-  if (warp == 0) {
+  if (warp == kProducerWarp) {
     if (lane == 0) {
       const CUtensorMap* mq = &maps.q[seq];
       const CUtensorMap* mk = &maps.k[seq];
@@ -111,61 +117,81 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       tma_prefetch_desc(mk);
       int stage = 0;
       uint32_t phase = 0;
+      int filled = 0;
       bool ok = true;
       for (int J = 0; J <= jmax && ok; ++J) {
         for (int t = 0; t < stages_per_tile && ok; ++t) {
           const int u = t / halves, hh = t % halves;
           if (!mbar_wait(&sm.empty[stage], phase ^ 1u, abort, args.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.full[stage], kStageBytes);
+          mbar_arrive_expect_tx(&sm.full[stage], (has1 ? 2 : 1) * kBytesA + kBytesB);
           uint8_t* sa = sm.stage[stage];
-          uint8_t* sb = sm.stage[stage] + kBytesA;
+          uint8_t* sb = sm.stage[stage] + 2 * kBytesA;
           const int ta = (I * kTileM) * s + u;
           const int tb = (J * kTileN) * s + (s - 1 - u);
-          for (int c = 0; c < loads_a; ++c)
-            tma_load_3d(sa + c * load_bytes, mq, &sm.full[stage], hh * 64, h, ta + c * rows_per_load * s);
+          for (int e = 0; e < (has1 ? 2 : 1); ++e)
+            for (int c = 0; c < loads_a; ++c)
+              tma_load_3d(sa + e * kBytesA + c * load_bytes, mq, &sm.full[stage], hh * 64, h0 + e,
+                          ta + c * rows_per_load * s);
           for (int c = 0; c < loads_b; ++c)
             tma_load_3d(sb + c * load_bytes, mk, &sm.full[stage], hh * 64, hk, tb + c * rows_per_load * s);
+          ++filled;
           if (++stage == kScoreStages) { stage = 0; phase ^= 1u; }
         }
       }
+      // every copy has landed before the CTA can exit (a stage holds at most
+      // one round in flight: the next round into it waits for its consumer)
+      for (int x = 0; x < kScoreStages && x < filled; ++x) {
+        const int last = filled - 1 - ((filled - 1 - x) % kScoreStages);  // last fill of stage x
+        mbar_wait_quiesce(&sm.full[x], (last / kScoreStages) & 1, args.status);
+      }
     }
     __syncwarp();
-  } else if (warp == 1) {
+  } else if (warp == kMmaWarp) {
     if (lane == 0) {
       const uint32_t idesc = make_idesc(kFp8 ? 0u : 1u, 0u, 128u, 256u);
+      const int nh = has1 ? 2 : 1;
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
       for (int J = 0; J <= jmax && ok; ++J) {
-        const int buf = J & 1;
-        const uint32_t acc_phase = (J >> 1) & 1;
-        if (!mbar_wait(&sm.acc_empty[buf], acc_phase ^ 1u, abort, args.status)) break;
-        tc_fence_after();
-        const uint32_t d_tmem = tmem + buf * 256;
         for (int t = 0; t < stages_per_tile; ++t) {
           if (!mbar_wait(&sm.full[stage], phase, abort, args.status)) { ok = false; break; }
           tc_fence_after();
           const uint32_t sa = smem_u32(sm.stage[stage]);
-          const uint32_t sb = sa + kBytesA;
+          const uint32_t sb = sa + 2 * kBytesA;
+          for (int e = 0; e < nh && ok; ++e) {
+            // a head's accumulator is overwritten from its first product of
+            // tile J on: its epilogue must have read tile J-1
+            if (t == 0) {
+              ok = mbar_wait(&sm.acc_empty[e], (J & 1) ^ 1u, abort, args.status);
+              if (!ok) break;
+              tc_fence_after();
+            }
+            const uint32_t d_tmem = tmem + 256 * e;
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk) {
-            const uint64_t ad = make_sdesc_sw128(sa + kk * 32, 16, 1024);
-            const uint64_t bd = make_sdesc_sw128(sb + kk * 32, 16, 1024);
-            if constexpr (kFp8) mma_f8_ss(d_tmem, ad, bd, idesc, (t | kk) != 0);
-            else mma_bf16_ss(d_tmem, ad, bd, idesc, (t | kk) != 0);
+            for (int kk = 0; kk < 4; ++kk) {
+              const uint64_t ad = make_sdesc_sw128(sa + e * kBytesA + kk * 32, 16, 1024);
+              const uint64_t bd = make_sdesc_sw128(sb + kk * 32, 16, 1024);
+              if constexpr (kFp8) mma_f8_ss(d_tmem, ad, bd, idesc, (t | kk) != 0);
+              else mma_bf16_ss(d_tmem, ad, bd, idesc, (t | kk) != 0);
+            }
           }
+          if (!ok) break;
           mma_commit(&sm.empty[stage]);
           if (++stage == kScoreStages) { stage = 0; phase ^= 1u; }
         }
-        if (ok) mma_commit(&sm.acc_full[buf]);
+        if (ok) mma_commit(&sm.acc_full);
       }
       // no MMA may still run when TMEM is released
       mma_commit(&sm.drain);
-      mbar_wait(&sm.drain, 0, abort, args.status);
+      mbar_wait_quiesce(&sm.drain, 0, args.status);
     }
     __syncwarp();
-  } else {
-    // epilogue: thread owns TMEM lane (query group of the tile) `row`
+  } else if (warp < 4 || has1) {
+    // epilogue: warpgroup e handles head h0 + e; thread owns TMEM lane (query
+    // group of the tile) `row`
+    const int e = warp >> 2;
+    const int h = h0 + e;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
     constexpr int gpb = kBlock / s;             // groups per block (16 for s = 8)
@@ -182,14 +208,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     constexpr int kbt = kTileN / gpb;    // key blocks per key tile (2 s)
     constexpr int kbc = 32 / gpb;        // key blocks per 32-column chunk
     for (int J = 0; J <= jmax; ++J) {
-      const int buf = J & 1;
       // every lane waits; the warp leaves together if any lane gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full[buf], (J >> 1) & 1, abort, args.status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full, J & 1, abort, args.status))) break;
       tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < 8; ++ch) {
         uint32_t r[32];
-        tmem_ld32(tmem + buf * 256 + ch * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r);
+        tmem_ld32(tmem + e * 256 + ch * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r);
         tmem_ld_wait();
         const int b0 = J * kTileN + ch * 32;  // first key group of the chunk
 #pragma unroll
@@ -209,7 +234,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+      if (lane == 0) mbar_arrive(&sm.acc_empty[e]);
       if (J == jmax && writer)
         for (int j = (jmax + 1) * kbt; j < args.nb_max; ++j) srow[j] = ninf;
     }
@@ -217,7 +242,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, kScoreTmemCols);
   }

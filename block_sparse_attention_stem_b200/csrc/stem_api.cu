@@ -217,7 +217,9 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   a.vbonus = vbonus;
   a.scores = scores;
   a.status = status;
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * ((si.nb + s - 1) / s); })) {
+  // one CTA per (pair of query heads of a KV group, 128-group query tile)
+  const int pairs = hkv * ((hq / hkv + 1) / 2);
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return pairs * ((si.nb + s - 1) / s); })) {
     ScoreMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {

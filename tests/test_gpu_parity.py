@@ -41,6 +41,7 @@ CASES = {
     "tiny_fp8": I.workload("tiny", dtype="fp8"),
     "varlen_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=16),
     "many_seqs": W([128 * (k % 5 + 1) + 8 * k for k in range(11)], 2, 1, seed=17),
+    "gqa3_odd_group": W([1500, 700], 6, 2, seed=18),  # three query heads per KV head
 }
 
 
