@@ -115,6 +115,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const CUtensorMap* mk = &maps.k[seq];
       tma_prefetch_desc(mq);
       tma_prefetch_desc(mk);
+      const bool grouped = maps.group_maps[seq] != 0;
+      const CUtensorMap* mqg = &maps.q_groups[seq];
+      const CUtensorMap* mkg = &maps.k_groups[seq];
+      if (grouped) {
+        tma_prefetch_desc(mqg);
+        tma_prefetch_desc(mkg);
+      }
+      // the partial last group (L % s tokens) lies outside the group maps
+      const int gpart = (L % s != 0) ? L / s : -1;
+      auto holds_partial = [&](int g0, int n) { return gpart >= g0 && gpart < g0 + n; };
+      const bool a_grouped = grouped && !holds_partial(I * kTileM, kTileM);
       int stage = 0;
       uint32_t phase = 0;
       int filled = 0;
@@ -128,12 +139,23 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
           uint8_t* sb = sm.stage[stage] + 2 * kBytesA;
           const int ta = (I * kTileM) * s + u;
           const int tb = (J * kTileN) * s + (s - 1 - u);
-          for (int e = 0; e < (has1 ? 2 : 1); ++e)
-            for (int c = 0; c < loads_a; ++c)
-              tma_load_3d(sa + e * kBytesA + c * load_bytes, mq, &sm.full[stage], hh * 64, h0 + e,
-                          ta + c * rows_per_load * s);
-          for (int c = 0; c < loads_b; ++c)
-            tma_load_3d(sb + c * load_bytes, mk, &sm.full[stage], hh * 64, hk, tb + c * rows_per_load * s);
+          // whole-group tiles: one copy per operand slab; the tile holding a
+          // partial last group: s-strided copies of 32 rows (zeros past the end)
+          if (a_grouped) {
+            for (int e = 0; e < (has1 ? 2 : 1); ++e)
+              tma_load_4d(sa + e * kBytesA, mqg, &sm.full[stage], hh * 64, h0 + e, u, I * kTileM);
+          } else {
+            for (int e = 0; e < (has1 ? 2 : 1); ++e)
+              for (int c = 0; c < loads_a; ++c)
+                tma_load_3d(sa + e * kBytesA + c * load_bytes, mq, &sm.full[stage], hh * 64, h0 + e,
+                            ta + c * rows_per_load * s);
+          }
+          if (grouped && !holds_partial(J * kTileN, kTileN)) {
+            tma_load_4d(sb, mkg, &sm.full[stage], hh * 64, hk, s - 1 - u, J * kTileN);
+          } else {
+            for (int c = 0; c < loads_b; ++c)
+              tma_load_3d(sb + c * load_bytes, mk, &sm.full[stage], hh * 64, hk, tb + c * rows_per_load * s);
+          }
           ++filled;
           if (++stage == kScoreStages) { stage = 0; phase ^= 1u; }
         }

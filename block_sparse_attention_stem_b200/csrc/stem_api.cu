@@ -171,6 +171,30 @@ EncodeTiledFn encode_fn() {
 
 // 3-D map over one sequence of a [T, H, 128] tensor: dims (d, head, token),
 // box (inner, 1, box_tokens) traversed with token stride `tstride`, 128-B swizzle.
+// The len / s full groups of s tokens of one sequence as a 4-d tensor
+// (dim, head, slot u, group g) -> token g s + u; box (one 128-B slab, 1, 1,
+// box_groups): one copy brings slot u of box_groups consecutive groups.  Only
+// whole groups are mapped, so no copy reads past the sequence; groups beyond
+// are zero-filled.  False when the sequence has no whole group.
+bool encode_group_map(CUtensorMap* m, const void* base, bool fp8, int heads, int tok0, int len, int s,
+                      int box_groups) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || len / s == 0) return false;
+  const size_t elt = fp8 ? 1 : 2;
+  const size_t row = static_cast<size_t>(heads) * kHeadDim * elt;  // bytes per token
+  const uint8_t* b = static_cast<const uint8_t*>(base) + static_cast<size_t>(tok0) * row;
+  cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                        static_cast<cuuint64_t>(s), static_cast<cuuint64_t>(len / s)};
+  cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim * elt), static_cast<cuuint64_t>(row),
+                           static_cast<cuuint64_t>(row * s)};
+  cuuint32_t box[4] = {static_cast<cuuint32_t>(fp8 ? 128 : 64), 1u, 1u, static_cast<cuuint32_t>(box_groups)};
+  cuuint32_t estr[4] = {1u, 1u, 1u, 1u};
+  CUresult r = fn(m, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+                  const_cast<uint8_t*>(b), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 bool encode_seq_map(CUtensorMap* m, const void* base, bool fp8, int heads, int tok0, int len, int box_tokens,
                     int tstride) {
   EncodeTiledFn fn = encode_fn();
@@ -225,6 +249,10 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
     for (int q = 0; q < b.n; ++q) {
       if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], 256, s) ||
           !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], 256, s))
+        return STEM_ERR_CUDA;
+      maps.group_maps[q] = b.len[q] / s > 0;
+      if (maps.group_maps[q] && (!encode_group_map(&maps.q_groups[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], s, 128) ||
+                                 !encode_group_map(&maps.k_groups[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], s, 256)))
         return STEM_ERR_CUDA;
     }
     stem_status_t st = cuda_status(launch_score(maps, b, a, fp8, stream));

@@ -15,6 +15,11 @@ namespace stem {
 struct ScoreMaps {
   CUtensorMap q[kMaxSeqPerLaunch];  // token traversal stride s, box 256 tokens
   CUtensorMap k[kMaxSeqPerLaunch];
+  // the full s-token groups of a sequence as (dim, head, slot, group), box of
+  // 128 (q) or 256 (k) groups of one slot; valid where group_maps[seq] != 0
+  CUtensorMap q_groups[kMaxSeqPerLaunch];
+  CUtensorMap k_groups[kMaxSeqPerLaunch];
+  int group_maps[kMaxSeqPerLaunch];
 };
 
 struct BsaMaps {
