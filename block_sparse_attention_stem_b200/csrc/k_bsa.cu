@@ -5,26 +5,25 @@
 // prepared outside it; a skipped block is the same as a block of -inf scores,
 // so the softmax needs no change; fixed 128 x 128 tiles).
 //
-// One CTA owns two CSR rows ("tiles"): consecutive rows of the KV-head-major,
-// longest-first order, i.e. the same query block of two query heads sharing a
-// KV head, whose budgets are equal.  Every listed key block j of a tile
+// One CTA owns one CSR row (a query block i of one query head); two CTAs run
+// on every SM, each with half of the SM's tensor memory, so the two rows
+// proceed independently and one CTA's start-up and epilogue overlap the other
+// CTA's main loop.  Rows are taken in KV-head-major, longest-first order, so
+// the CTAs in flight share one KV head's K/V in L2.  Every listed key block j
 // (ascending, the diagonal last) is processed as two halves of 64 keys,
 // h = 2n and 2n + 1:
 //   S_h = Q K_h^T          tcgen05.mma (M 128, N 64), Q and K from SMEM, fp32
-//                          into S buffer h % 2 of the tile (TMEM)
-//   P_h = exp2(S_h c - m)  the tile's softmax warpgroup (thread = query row =
-//                          TMEM lane); P is written back over S_h
+//                          into S buffer h % 2 (TMEM)
+//   P_h = exp2(S_h c - m)  the softmax warpgroup (thread = query row = TMEM
+//                          lane); P is written back over S_h
 //   O += P_h V_h           tcgen05.mma with P from TMEM, V from SMEM
 //                          (MN-major); the fp32 accumulator stays in TMEM
-// With two S buffers per tile, S_{h+1} is computed while the softmax of half
-// h runs, so the softmax never waits for the tensor core; the tensor core
-// takes the products of whichever tile is ready (each tile has its own TMA
-// producer and its own MMA issuer).  Both tiles' softmax warps share the
-// SM's exp2 units, which keeps those units busy.
+// With two S buffers, S_{h+1} is computed while the softmax of half h runs, so
+// the softmax does not wait for the tensor core in steady state.
 // The reference row max m moves (and O is rescaled in TMEM) only when a half
 // raises it past a threshold (2^8 bf16, 2^1 fp8), so P stays bounded and
 // rescales are rare; O and the row sum share that reference, so the result is
-// exact.  A rescale first waits for P_{h-1} V_{h-1} (S_h no longer implies it).
+// exact.  A rescale first waits for P_{h-1} V_{h-1} (S_h does not imply it).
 // Masking happens only on the diagonal block.
 //
 // fp8: a single e4m3 P carries three mantissa bits (up to 6% error per weight,
@@ -36,18 +35,15 @@
 // goes to columns 16ch..16ch+15 of the S buffer (bf16 pairs, or 8 columns of
 // hi and 8 of lo for e4m3); the whole half is in registers by then.
 //
-// Warp roles (448 threads):
-//   warps 0-3    softmax + epilogue of tile 0 (TMEM lane quarters 0-3)
-//   warps 4-7    softmax + epilogue of tile 1
-//   warps 8-11   TMA producers: tile 0 Q and K, tile 0 V, tile 1 Q and K,
-//                tile 1 V (64-key halves)
-//   warps 12, 13 MMA issuer of tile 0, 1 (warp 12 owns the TMEM allocation)
-// Each tile has two K slots and two V slots (half h uses slot h % 2).  The
-// completion of S_h frees K slot h % 2 and that of P_h V_h frees V slot h % 2,
-// so a product needs one commit.  Tile 1 starts once tile 0 has stored its
-// first P, which staggers the two softmax warpgroups: while one computes
-// exponentials the other is in its row-max and bookkeeping phase.
-// Block lists are staged in shared memory; every wait is bounded.
+// Warp roles (224 threads):
+//   warps 0-3  softmax + epilogue (TMEM lane quarters 0-3)
+//   warp  4    TMA producer of Q and the K halves (and stages the block list)
+//   warp  5    TMA producer of the V halves (one issuing thread moves only
+//              about 26 B per cycle, so K and V get a thread each)
+//   warp  6    TMEM owner and MMA issuer
+// Half h uses K slot and V slot h % 2: K_{h+2} may overwrite K_h once S_h is
+// complete, V_{h+2} may overwrite V_h once P_h V_h is, so a product needs one
+// commit.  Block lists are staged in shared memory; every wait is bounded.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
 
@@ -55,10 +51,11 @@ namespace stem {
 
 namespace {
 
-constexpr int kBsaThreads = 448;
-constexpr int kProducerWarp = 8;  // + 2 tile + (0: Q and K, 1: V)
-constexpr int kMmaWarp = 12;      // + tile; warp 12 owns TMEM
-constexpr uint32_t kBsaTmemCols = 512;  // tile t: S buffers at 256 t and 256 t + 64, O at 256 t + 128
+constexpr int kBsaThreads = 224;
+constexpr int kKProducerWarp = 4;
+constexpr int kVProducerWarp = 5;
+constexpr int kMmaWarp = 6;
+constexpr uint32_t kBsaTmemCols = 256;  // S buffers at 0 and 64, O at 128
 constexpr int kHalf = 64;               // keys per S buffer
 constexpr int kMaxList = 2048;          // list entries per tile staged in SMEM
 // Pairs of keys (bit k: keys 2k, 2k+1 of a 32-key chunk) whose exp2 runs on
@@ -79,21 +76,20 @@ template struct BsaCfg<true>;
 
 template <bool kFp8>
 struct BsaSmem {
-  uint8_t q[2][BsaCfg<kFp8>::kQBytes];                                   // 1024-aligned
-  uint8_t k[2][2][BsaCfg<kFp8>::kHalfBytes];  // per tile, per slot
-  uint8_t v[2][2][BsaCfg<kFp8>::kHalfBytes];
-  uint64_t q_full[2];
-  uint64_t k_full[2][2];  // per tile and slot: K_h landed
-  uint64_t v_full[2][2];  // per tile and slot: V_h landed
-  uint64_t s_full[2][2];  // per tile and S buffer: S_h complete (K slot free again)
-  uint64_t v_free[2][2];  // per tile and slot: P_h V_h complete (V slot free again)
-  uint64_t p_full[2][2];  // per tile and S buffer: 4 softmax warps stored P_h (and rescaled O)
-  uint64_t o_done[2];     // per tile: the last P V is complete
-  uint64_t drain[2];      // per tile: every MMA of that tile's issuer complete
-  uint64_t stagger;       // tile 0 stored its first P
-  int32_t list[2][kMaxList];
-  int nvalid[2];
-  int in_smem[2];
+  uint8_t q[BsaCfg<kFp8>::kQBytes];                        // 1024-aligned
+  uint8_t k[2][BsaCfg<kFp8>::kHalfBytes];                  // per slot
+  uint8_t v[2][BsaCfg<kFp8>::kHalfBytes];
+  uint64_t q_full;
+  uint64_t k_full[2];  // per slot: K_h landed
+  uint64_t v_full[2];  // per slot: V_h landed
+  uint64_t s_full[2];  // per S buffer: S_h complete (K slot free again)
+  uint64_t v_free[2];  // per slot: P_h V_h complete (V slot free again)
+  uint64_t p_full[2];  // per S buffer: the 4 softmax warps stored P_h (and rescaled O)
+  uint64_t o_done;     // the last P V is complete
+  uint64_t drain;      // every MMA of the issuer complete
+  int32_t list[kMaxList];
+  int nvalid;
+  int in_smem;
   uint32_t tmem_base;
   int abort;
 };
@@ -193,7 +189,7 @@ __device__ __forceinline__ void exp_chunk_bf16(const uint32_t* rr, float2 c2, fl
 }  // namespace
 
 template <bool kFp8>
-__global__ void __launch_bounds__(kBsaThreads, 1)
+__global__ void __launch_bounds__(kBsaThreads, 2)
     bsa_kernel(const __grid_constant__ BsaMaps maps, const SeqBatch batch, const BsaArgs args) {
   using Cfg = BsaCfg<kFp8>;
   constexpr int kSlabs = kFp8 ? 1 : 2;  // 128-byte head-dim slabs per row (bf16: dims 0-63 and 64-127)
@@ -203,46 +199,37 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
 
   const int warp = warp_id(), lane = lane_id();
   const int seq = find_seq(batch, blockIdx.x);
-  const int pair = blockIdx.x - batch.item0[seq];
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
   const int G = args.hq / args.hkv;
-  Tile tile[2];
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    // Rows of a sequence in KV-head-major order: KV head, then query blocks
-    // descending (longest rows first), then the query heads of the group.
-    // CTAs in flight then share one KV head's K/V, which fits in L2.
-    const int item = 2 * pair + t;
-    tile[t].valid = item < args.hq * nb;
-    const int it = tile[t].valid ? item : 0;
+  // Rows of a sequence in KV-head-major order: KV head, then query blocks
+  // descending (longest rows first), then the query heads of the group.
+  Tile tl;
+  {
+    const int it = blockIdx.x - batch.item0[seq];
     const int hk_of = it / (G * nb);
     const int rem = it % (G * nb);
-    tile[t].i = nb - 1 - rem / G;
-    tile[t].h = hk_of * G + rem % G;
-    tile[t].hk = tile[t].h / G;
-    const size_t r = static_cast<size_t>(tile[t].h) * args.nbtot + batch.g0[seq] + tile[t].i;
-    tile[t].beg = tile[t].valid ? args.row_ptr[r] : 0;
-    tile[t].end = tile[t].valid ? args.row_ptr[r + 1] : 0;
+    tl.valid = true;
+    tl.i = nb - 1 - rem / G;
+    tl.h = hk_of * G + rem % G;
+    tl.hk = tl.h / G;
+    const size_t r = static_cast<size_t>(tl.h) * args.nbtot + batch.g0[seq] + tl.i;
+    tl.beg = args.row_ptr[r];
+    tl.end = args.row_ptr[r + 1];
   }
 
-  if (warp == kProducerWarp) stage_list(args.col_idx, tile[0], sm.list[0], &sm.nvalid[0], &sm.in_smem[0], args.status);
-  if (warp == kProducerWarp + 2)
-    stage_list(args.col_idx, tile[1], sm.list[1], &sm.nvalid[1], &sm.in_smem[1], args.status);
+  if (warp == kKProducerWarp) stage_list(args.col_idx, tl, sm.list, &sm.nvalid, &sm.in_smem, args.status);
   if (threadIdx.x == 0) {
-    for (int t = 0; t < 2; ++t) {
-      mbar_init(&sm.q_full[t], 1);
-      for (int b = 0; b < 2; ++b) {
-        mbar_init(&sm.k_full[t][b], 1);
-        mbar_init(&sm.v_full[t][b], 1);
-        mbar_init(&sm.s_full[t][b], 1);
-        mbar_init(&sm.v_free[t][b], 1);
-        mbar_init(&sm.p_full[t][b], 4);
-      }
-      mbar_init(&sm.o_done[t], 1);
-      mbar_init(&sm.drain[t], 1);
+    mbar_init(&sm.q_full, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.k_full[b], 1);
+      mbar_init(&sm.v_full[b], 1);
+      mbar_init(&sm.s_full[b], 1);
+      mbar_init(&sm.v_free[b], 1);
+      mbar_init(&sm.p_full[b], 4);
     }
-    mbar_init(&sm.stagger, 1);
+    mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
   }
@@ -254,41 +241,32 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
-  const int nv[2] = {sm.nvalid[0], sm.nvalid[1]};
-  const bool lsm[2] = {sm.in_smem[0] != 0, sm.in_smem[1] != 0};
+  const int N = sm.nvalid;
+  const bool list_in_smem = sm.in_smem != 0;
   volatile int* abort = &sm.abort;
 
-  if (warp >= kProducerWarp && warp < kProducerWarp + 4) {
+  if (warp == kKProducerWarp || warp == kVProducerWarp) {
     // ------------------------------------------------------------ producers
-    // warp 8 + 2 t + kind: kind 0 loads Q and the K halves of tile t, kind 1
-    // the V halves (one issuing thread moves only about 26 B per cycle, so
-    // K and V get a thread each)
-    const int t = (warp - kProducerWarp) >> 1;
-    const bool is_v = ((warp - kProducerWarp) & 1) != 0;
-    const Tile tl = (t == 0) ? tile[0] : tile[1];
-    const int N = (t == 0) ? nv[0] : nv[1];
+    const bool is_v = warp == kVProducerWarp;
     if (lane == 0 && N > 0) {
-      const bool list_in_smem = (t == 0) ? lsm[0] : lsm[1];
       const CUtensorMap* m = is_v ? &maps.v[seq] : &maps.k[seq];
       tma_prefetch_desc(m);
       if (!is_v) {
-        mbar_arrive_expect_tx(&sm.q_full[t], Cfg::kQBytes);
+        mbar_arrive_expect_tx(&sm.q_full, Cfg::kQBytes);
         for (int hh = 0; hh < kSlabs; ++hh)
-          tma_load_3d(sm.q[t] + hh * 16384, &maps.q[seq], &sm.q_full[t], hh * 64, tl.h, tl.i * kBlock);
+          tma_load_3d(sm.q + hh * 16384, &maps.q[seq], &sm.q_full, hh * 64, tl.h, tl.i * kBlock);
       }
-      // Half h goes to slot h % 2.  K_{h+2} may overwrite K_h once S_h is
-      // complete, V_{h+2} may overwrite V_h once P_h V_h is.
       const int H = 2 * N;
       ListCursor cur(tl.beg);
       int j = 0, issued = 0;
       for (int h = 0; h < H; ++h) {
         if (h >= 2) {
-          uint64_t* freed = is_v ? &sm.v_free[t][h & 1] : &sm.s_full[t][h & 1];
+          uint64_t* freed = is_v ? &sm.v_free[h & 1] : &sm.s_full[h & 1];
           if (!mbar_wait(freed, ((h - 2) >> 1) & 1, abort, args.status)) break;
         }
-        if ((h & 1) == 0) j = cur.next(sm.list[t], list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
-        uint8_t* dst = is_v ? sm.v[t][h & 1] : sm.k[t][h & 1];
-        uint64_t* bar = is_v ? &sm.v_full[t][h & 1] : &sm.k_full[t][h & 1];
+        if ((h & 1) == 0) j = cur.next(sm.list, list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
+        uint8_t* dst = is_v ? sm.v[h & 1] : sm.k[h & 1];
+        uint64_t* bar = is_v ? &sm.v_full[h & 1] : &sm.k_full[h & 1];
         mbar_arrive_expect_tx(bar, Cfg::kHalfBytes);
         for (int hh = 0; hh < kSlabs; ++hh)
           tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, j * kBlock + (h & 1) * kHalf);
@@ -297,28 +275,26 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
       // every copy of this producer has landed before the CTA can exit (a
       // slot holds at most one copy in flight: the next copy into it waits
       // for the product that consumes this one)
-      if (!is_v) mbar_wait_quiesce(&sm.q_full[t], 0, args.status);
+      if (!is_v) mbar_wait_quiesce(&sm.q_full, 0, args.status);
       for (int x = 0; x < 2 && x < issued; ++x) {
         const int last = issued - 1 - ((issued - 1 - x) & 1);  // last half issued into slot x
-        mbar_wait_quiesce(is_v ? &sm.v_full[t][x] : &sm.k_full[t][x], (last >> 1) & 1, args.status);
+        mbar_wait_quiesce(is_v ? &sm.v_full[x] : &sm.k_full[x], (last >> 1) & 1, args.status);
       }
     }
     __syncwarp();
-  } else if (warp == kMmaWarp || warp == kMmaWarp + 1) {
-    // ------------------------------------------------------------ MMA issuer of tile t
-    const int t = warp - kMmaWarp;
-    const int N = (t == 0) ? nv[0] : nv[1];
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && N > 0) {
       const uint32_t idesc_s = make_idesc(kFp8 ? 0u : 1u, 0u, 128u, static_cast<uint32_t>(kHalf));
       const uint32_t idesc_o = make_idesc(kFp8 ? 0u : 1u, 1u, 128u, 128u);
-      const uint32_t sq = smem_u32(sm.q[t]);
-      const uint32_t o_tmem = tmem + 256 * t + 128;
+      const uint32_t sq = smem_u32(sm.q);
+      const uint32_t o_tmem = tmem + 128;
       const int H = 2 * N;
       auto issue_s = [&](int h) -> bool {  // S_h = Q K_h^T into buffer h % 2
-        if (!mbar_wait(&sm.k_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        if (!mbar_wait(&sm.k_full[h & 1], (h >> 1) & 1, abort, args.status)) return false;
         tc_fence_after();
-        const uint32_t sk = smem_u32(sm.k[t][h & 1]);
-        const uint32_t d = tmem + 256 * t + kHalf * (h & 1);
+        const uint32_t sk = smem_u32(sm.k[h & 1]);
+        const uint32_t d = tmem + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // 32 head dims per step
@@ -330,15 +306,15 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
             mma_bf16_ss(d, make_sdesc_sw128(sq + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
                         make_sdesc_sw128(sk + (kk >> 2) * (kHalf * 128) + (kk & 3) * 32, 16, 1024), idesc_s, kk != 0);
         }
-        mma_commit(&sm.s_full[t][h & 1]);
+        mma_commit(&sm.s_full[h & 1]);
         return true;
       };
       auto issue_pv = [&](int h) -> bool {  // O += P_h V_h
-        if (!mbar_wait(&sm.p_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
-        if (!mbar_wait(&sm.v_full[t][h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        if (!mbar_wait(&sm.p_full[h & 1], (h >> 1) & 1, abort, args.status)) return false;
+        if (!mbar_wait(&sm.v_full[h & 1], (h >> 1) & 1, abort, args.status)) return false;
         tc_fence_after();
-        const uint32_t sv = smem_u32(sm.v[t][h & 1]);
-        const uint32_t p = tmem + 256 * t + kHalf * (h & 1);
+        const uint32_t sv = smem_u32(sm.v[h & 1]);
+        const uint32_t p = tmem + kHalf * (h & 1);
         if constexpr (kFp8) {
 #pragma unroll
           for (int kk = 0; kk < 2; ++kk)        // 32 keys per step
@@ -352,53 +328,47 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
             mma_bf16_ts(o_tmem, p + kk * 8, make_sdesc_sw128(sv + kk * 2048, kHalf * 128, 1024), idesc_o,
                         (h | kk) != 0);
         }
-        mma_commit(&sm.v_free[t][h & 1]);
-        if (h == H - 1) mma_commit(&sm.o_done[t]);
+        mma_commit(&sm.v_free[h & 1]);
+        if (h == H - 1) mma_commit(&sm.o_done);
         return true;
       };
-      // tile 1 starts once tile 0 stored its first P (see the header)
-      bool ok = !(t == 1 && nv[0] > 0) || mbar_wait(&sm.stagger, 0, abort, args.status);
       // S_0, S_1, then per half h: P_h V_h and S_{h+2} (into the buffer P_h
-      // V_h just read: one issuer's products run in order)
-      ok = ok && mbar_wait(&sm.q_full[t], 0, abort, args.status) && issue_s(0) && issue_s(1);
+      // V_h just read: the tensor core runs one issuer's products in order)
+      bool ok = mbar_wait(&sm.q_full, 0, abort, args.status) && issue_s(0) && issue_s(1);
       for (int h = 0; h < H && ok; ++h) {
         ok = issue_pv(h);
         if (ok && h + 2 < H) ok = issue_s(h + 2);
       }
-      // no MMA of this issuer may still run when TMEM is released
-      mma_commit(&sm.drain[t]);
-      mbar_wait_quiesce(&sm.drain[t], 0, args.status);
+      // no MMA may still run when TMEM is released
+      mma_commit(&sm.drain);
+      mbar_wait_quiesce(&sm.drain, 0, args.status);
     }
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax + epilogue
-    const int t = warp >> 2;   // tile of this warpgroup
-    const int q4 = warp & 3;   // TMEM lane quarter
+    const int q4 = warp;  // TMEM lane quarter
     const int row = q4 * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(q4 * 32) << 16;
-    const Tile tl = (t == 0) ? tile[0] : tile[1];  // per-field selects, no local-memory indexing
-    const int N = (t == 0) ? nv[0] : nv[1];
-    const bool list_in_smem = (t == 0) ? lsm[0] : lsm[1];
     const int t_row = tl.i * kBlock + row;  // token of this row inside the sequence
     const size_t tok = static_cast<size_t>(batch.tok0[seq]) + t_row;
     float c = args.scale_log2;  // sigma * log2(e) (* q_scale * k_scale for fp8)
     if constexpr (kFp8) c *= args.q_scale[tl.h] * args.k_scale[tl.hk];
     const float ninf = -__int_as_float(0x7f800000);
-    const uint32_t s_base = tmem + 256 * t + lane_off;
-    const uint32_t o_tmem = tmem + 256 * t + 128 + lane_off;
+    const uint32_t s_base = tmem + lane_off;
+    const uint32_t o_tmem = tmem + 128 + lane_off;
 
     float m_ref = ninf;  // reference max (scaled log2 domain) shared by O and l
     float l = 0.f;       // row sum of exp2(s c - m_ref)
     bool ok = true;
     ListCursor cur(tl.beg);
     for (int n = 0; n < N && ok; ++n) {
-      const int j = cur.next(sm.list[t], list_in_smem, n, args.col_idx, tl.end, tl.i);
+      const int j = cur.next(sm.list, list_in_smem, n, args.col_idx, tl.end, tl.i);
       const bool diag = (j == tl.i);
 #pragma unroll 1
       for (int half = 0; half < 2; ++half) {
         const int h = 2 * n + half;
         const uint32_t s_tmem = s_base + kHalf * half;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[t][half], n & 1, abort, args.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[half], n & 1, abort, args.status))) {
           ok = false;
           break;
         }
@@ -438,7 +408,7 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
           if (h >= 1) {
             // O holds P V up to half h-1: let that product finish first
             if (!__all_sync(0xffffffffu,
-                            mbar_wait(&sm.v_free[t][(h - 1) & 1], ((h - 1) >> 1) & 1, abort, args.status))) {
+                            mbar_wait(&sm.v_free[(h - 1) & 1], ((h - 1) >> 1) & 1, abort, args.status))) {
               ok = false;
               break;
             }
@@ -499,15 +469,14 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.p_full[t][half]);
-        if (t == 0 && h == 0 && warp == 0 && lane == 0) mbar_arrive(&sm.stagger);
+        if (lane == 0) mbar_arrive(&sm.p_full[half]);
       }
     }
 
     // epilogue: normalise O and store this row (the TMEM reads are warp-wide;
     // only rows inside the sequence are stored)
-    if (tl.valid) {
-      const bool have_o = ok && N > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.o_done[t], 0, abort, args.status));
+    {
+      const bool have_o = ok && N > 0 && __all_sync(0xffffffffu, mbar_wait(&sm.o_done, 0, abort, args.status));
       if (have_o) tc_fence_after();
       const bool store = t_row < L;
       float inv = (l > 0.f) ? 1.f / l : 0.f;
@@ -546,7 +515,12 @@ __global__ void __launch_bounds__(kBsaThreads, 1)
   }
 }
 
-size_t bsa_smem_bytes(bool fp8) { return (fp8 ? sizeof(BsaSmem<true>) : sizeof(BsaSmem<false>)) + 1024; }
+// At least 80 KB, so that no more than two CTAs share an SM's tensor memory
+// (each allocates half of it; a third would wait in tcgen05.alloc).
+size_t bsa_smem_bytes(bool fp8) {
+  const size_t need = (fp8 ? sizeof(BsaSmem<true>) : sizeof(BsaSmem<false>)) + 1024;
+  return need > (size_t(80) << 10) ? need : (size_t(80) << 10);
+}
 
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
                        cudaStream_t stream) {

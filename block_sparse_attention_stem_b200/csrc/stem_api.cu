@@ -298,8 +298,8 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.out = out;
   a.lse = lse;
   a.status = status;
-  // one CTA per pair of consecutive rows (same query block, neighbouring heads)
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return (hq * si.nb + 1) / 2; })) {
+  // one CTA per CSR row (query head, query block)
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
     BsaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
