@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "STEM_OK", 1: "STEM_ERR_INVALID_ARG", 2: "STEM_ERR_UNSUPPORTE
                 3: "STEM_ERR_WORKSPACE_TOO_SMALL", 4: "STEM_ERR_MISALIGNED", 5: "STEM_ERR_CUDA",
                 6: "STEM_ERR_TIMEOUT", 7: "STEM_ERR_BAD_BLOCKLIST"}
 STEM_BF16, STEM_FP8_E4M3 = 0, 1
-EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill", "stem_prefill_noalloc",
+EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill", "stem_prefill_host",
+            "stem_prefill_noalloc",
             "stem_selftest_wait_timeout", "stem_read_device_status", "stem_status_string", "stem_version")
 
 
@@ -70,6 +71,7 @@ def _load() -> ctypes.CDLL:
     lib.stem_bsa_fwd.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill_noalloc.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp]
+    lib.stem_prefill_host.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.stem_selftest_wait_timeout.argtypes = [vp, vp]
     lib.stem_read_device_status.argtypes = [vp, vp, P(ctypes.c_int)]
     lib.stem_status_string.argtypes = [ctypes.c_int]
@@ -223,6 +225,32 @@ def stem_prefill(qkv: QKV, params: StemParams, out=None, lse=None, row_ptr=None,
     _check(LIB.stem_prefill(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(out), _ptr(lse), _ptr(row_ptr),
                             _ptr(col_idx), _ptr(ws), ws.numel(), _stream(stream)), "stem_prefill")
     return out, lse, row_ptr, (None if col_idx is None else col_idx[:pl.nnz]), ws
+
+
+def stem_prefill_host(qkv: QKV, params: StemParams, q_host, k_host, v_host, out_host, lse_host, out=None, lse=None,
+                      ws=None, stream=None):
+    """stem_prefill with inputs and outputs in (page-locked) host tensors; the
+    device tensors of `qkv` are filled by the call, transfers overlap compute.
+    Only enqueues: synchronize `stream` before reading out_host / lse_host."""
+    pl = stem_plan(qkv, params)
+    dev = qkv.q.device
+    T, hq = qkv.total_tokens, qkv.q.shape[1]
+    for name, t, like in (("q_host", q_host, qkv.q), ("k_host", k_host, qkv.k), ("v_host", v_host, qkv.v)):
+        if t.device.type != "cpu" or t.shape != like.shape or t.dtype != like.dtype or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous host tensor shaped like the device one")
+    if out_host.device.type != "cpu" or tuple(out_host.shape) != (T, hq, 128) or out_host.dtype != torch.bfloat16:
+        raise ValueError("out_host must be a host bf16 tensor [T, Hq, 128]")
+    if lse_host.device.type != "cpu" or tuple(lse_host.shape) != (hq, T) or lse_host.dtype != torch.float32:
+        raise ValueError("lse_host must be a host fp32 tensor [Hq, T]")
+    if out is None:
+        out = torch.empty(T, hq, 128, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    ws = _ws(pl.ws_prefill_bytes, dev, ws)
+    _check(LIB.stem_prefill_host(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(q_host), _ptr(k_host),
+                                 _ptr(v_host), _ptr(out), _ptr(lse), _ptr(out_host), _ptr(lse_host), _ptr(ws),
+                                 ws.numel(), _stream(stream)), "stem_prefill_host")
+    return out, lse, ws
 
 
 def stem_prefill_noalloc(qkv: QKV, params: StemParams, out=None, lse=None, row_ptr=None, col_idx=None,

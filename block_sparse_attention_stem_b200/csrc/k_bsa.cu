@@ -207,7 +207,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
   Tile tl;
   {
     const int it = blockIdx.x - batch.item0[seq];
-    const int hk_of = it / (G * nb);
+    const int hk_of = args.hk0 + it / (G * nb);
     const int rem = it % (G * nb);
     tl.valid = true;
     tl.i = nb - 1 - rem / G;

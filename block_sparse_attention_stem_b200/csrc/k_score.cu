@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   // group) so the CTAs in flight share one KV head's keys in L2.
   const int G = args.hq / args.hkv;
   const int npair = (G + 1) / 2;
-  const int hk = local / (npair * ntile);
+  const int hk = args.hk0 + local / (npair * ntile);
   const int rem = local % (npair * ntile);
   const int I = ntile - 1 - rem / npair;  // longest rows first within a KV head
   const int h0 = hk * G + 2 * (rem % npair);

@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const SeqBatch b
       static_cast<int32_t>(static_cast<int64_t>(hq) * nnz_per_head);
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batch, int hq, int nbtot, int nb_max,
-                                                             int sink, int window,
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batch, int h0, int nh, int nbtot,
+                                                             int nb_max, int sink, int window,
                                                              const float* __restrict__ scores,
                                                              const int32_t* __restrict__ budgets,
                                                              const int32_t* __restrict__ row_ptr,
@@ -106,9 +106,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batc
   const int s = find_seq(batch, blockIdx.x);
   const int local = blockIdx.x - batch.item0[s];
   const int nb = batch.nb[s];
-  // rows of a sequence: query blocks descending (longest rows first), heads inner
-  const int h = local % hq;
-  const int i = nb - 1 - local / hq;
+  // rows of a sequence: query blocks descending (longest rows first), heads
+  // h0 .. h0 + nh - 1 inner
+  const int h = h0 + local % nh;
+  const int i = nb - 1 - local / nh;
   const int g = batch.g0[s] + i;
   const size_t r = static_cast<size_t>(h) * nbtot + g;
   const int c = i + 1;
@@ -211,18 +212,18 @@ cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const SeqBatch& batch, int hq, int nbtot, int nb_max, int sink, int window,
+cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int nbtot, int nb_max, int sink, int window,
                           const float* scores, const int32_t* budgets, const int32_t* row_ptr, int32_t* col_idx,
                           cudaStream_t stream) {
   const int items = batch.item0[batch.n];
-  if (items == 0) return cudaSuccess;
+  if (items == 0 || nh <= 0 || h0 < 0 || h0 + nh > hq) return items == 0 || nh <= 0 ? cudaSuccess : cudaErrorInvalidValue;
   const size_t smem = sizeof(uint32_t) * static_cast<size_t>(nb_max);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  select_kernel<<<items, kSelThreads, smem, stream>>>(batch, hq, nbtot, nb_max, sink, window, scores, budgets,
+  select_kernel<<<items, kSelThreads, smem, stream>>>(batch, h0, nh, nbtot, nb_max, sink, window, scores, budgets,
                                                       row_ptr, col_idx);
   return cudaGetLastError();
 }

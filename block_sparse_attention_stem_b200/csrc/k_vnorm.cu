@@ -17,19 +17,19 @@ namespace stem {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const uint8_t* __restrict__ v,
-                                                    const float* __restrict__ v_scale, int hkv, int nbtot,
-                                                    float beta, float* __restrict__ vbonus) {
-  extern __shared__ unsigned int s_max[];  // [hkv] bit patterns of non-negative floats
+                                                    const float* __restrict__ v_scale, int hkv, int hk0, int nhk,
+                                                    int nbtot, float beta, float* __restrict__ vbonus) {
+  extern __shared__ unsigned int s_max[];  // [nhk] bit patterns of non-negative floats (KV heads hk0 ..)
   const int s = find_seq(batch, blockIdx.x);
   const int j = blockIdx.x - batch.item0[s];
   const int t0 = j * kBlock;
   const int ntok = min(kBlock, batch.len[s] - t0);
-  for (int h = threadIdx.x; h < hkv; h += blockDim.x) s_max[h] = 0u;
+  for (int h = threadIdx.x; h < nhk; h += blockDim.x) s_max[h] = 0u;
   __syncthreads();
 
   constexpr int kElt = kFp8 ? 1 : 2;
   constexpr int kLanesPerRow = (kHeadDim * kElt) / 16;  // 16-byte vectors per row: 16 (bf16) or 8 (fp8)
-  const int rows = ntok * hkv;
+  const int rows = ntok * nhk;  // (token, head) rows of this block and head range
   const int sub = threadIdx.x % kLanesPerRow;
   const int row_step = blockDim.x / kLanesPerRow;
   const uint8_t* base = v + (static_cast<size_t>(batch.tok0[s]) + t0) * hkv * kHeadDim * kElt;
@@ -38,7 +38,8 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
     float acc = 0.f;
     const bool valid = r0 < rows;
     if (valid) {
-      const uint4 w = *reinterpret_cast<const uint4*>(base + static_cast<size_t>(r0) * kHeadDim * kElt + sub * 16);
+      const size_t row = static_cast<size_t>(r0 / nhk) * hkv + hk0 + r0 % nhk;
+      const uint4 w = *reinterpret_cast<const uint4*>(base + row * kHeadDim * kElt + sub * 16);
       const uint32_t u[4] = {w.x, w.y, w.z, w.w};
       if constexpr (!kFp8) {
 #pragma unroll
@@ -66,31 +67,31 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
 #pragma unroll
     for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
     if (valid && sub == 0) {
-      const int h = r0 % hkv;
-      if constexpr (kFp8) acc *= v_scale[h] * v_scale[h];
+      const int h = r0 % nhk;
+      if constexpr (kFp8) acc *= v_scale[hk0 + h] * v_scale[hk0 + h];
       atomicMax(&s_max[h], __float_as_uint(acc));
     }
   }
   __syncthreads();
   const int g = batch.g0[s] + j;
-  for (int h = threadIdx.x; h < hkv; h += blockDim.x) {
+  for (int h = threadIdx.x; h < nhk; h += blockDim.x) {
     const float m = __uint_as_float(s_max[h]);
     const float lg = logf(m);  // ln 0 = -inf -> bonus 0
-    vbonus[static_cast<size_t>(h) * nbtot + g] = beta * fmaxf(0.f, lg);
+    vbonus[static_cast<size_t>(hk0 + h) * nbtot + g] = beta * fmaxf(0.f, lg);
   }
 }
 
-cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv,
-                         int nbtot, float beta, float* vbonus, cudaStream_t stream) {
+cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
+                         int nhk, int nbtot, float beta, float* vbonus, cudaStream_t stream) {
   const int items = batch.item0[batch.n];
-  if (items == 0) return cudaSuccess;
-  const size_t smem = sizeof(unsigned int) * static_cast<size_t>(hkv);
+  if (items == 0 || nhk <= 0) return cudaSuccess;
+  const size_t smem = sizeof(unsigned int) * static_cast<size_t>(nhk);
   if (fp8)
-    vnorm_kernel<true><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, nbtot,
-                                                     beta, vbonus);
+    vnorm_kernel<true><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
+                                                     nbtot, beta, vbonus);
   else
-    vnorm_kernel<false><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, nbtot,
-                                                      beta, vbonus);
+    vnorm_kernel<false><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
+                                                      nbtot, beta, vbonus);
   return cudaGetLastError();
 }
 

@@ -219,14 +219,16 @@ double sm_scale(const stem_params_t* p) {
 }
 
 // ---------------------------------------------------------------- stages
-stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, float* scores,
+// Every run_* below handles the KV heads hk0 .. hk0 + nhk - 1 (and their query
+// heads) only, so a caller can work through a layer one KV-head group at a time.
+stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk, float* scores,
                         float* vbonus, int* status, cudaStream_t stream) {
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads, s = p->stride;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
   for (const SeqBatch& b : make_batches(pl, [](const SeqInfo& si) { return si.nb; })) {
     stem_status_t st = cuda_status(
-        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, nbtot, static_cast<float>(p->beta), vbonus, stream));
+        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, hk0, nhk, nbtot, static_cast<float>(p->beta), vbonus, stream));
     if (st != STEM_OK) return st;
   }
   ScoreArgs a{};
@@ -241,8 +243,9 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   a.vbonus = vbonus;
   a.scores = scores;
   a.status = status;
+  a.hk0 = hk0;
   // one CTA per (pair of query heads of a KV group, 128-group query tile)
-  const int pairs = hkv * ((hq / hkv + 1) / 2);
+  const int pairs = nhk * ((hq / hkv + 1) / 2);
   for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return pairs * ((si.nb + s - 1) / s); })) {
     ScoreMaps maps;
     std::memset(&maps, 0, sizeof(maps));
@@ -261,25 +264,30 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   return STEM_OK;
 }
 
-stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, const float* scores,
+stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
+                         bool with_budgets, const float* scores,
                          int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, cudaStream_t stream) {
   const int hq = qkv->num_q_heads;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
+  const int G = hq / qkv->num_kv_heads;
   for (const SeqBatch& b : make_batches(pl, [](const SeqInfo&) { return 1; })) {
+    if (!with_budgets) break;
     stem_status_t st = cuda_status(launch_budget(b, hq, nbtot, pl.pub.nnz_per_head, p->keep_ratio, p->mu,
                                                  p->sink_blocks, p->window_blocks, p->budget_mode, budgets,
                                                  row_ptr, stream));
     if (st != STEM_OK) return st;
   }
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
-    stem_status_t st = cuda_status(launch_select(b, hq, nbtot, nb_max, p->sink_blocks, p->window_blocks, scores,
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * G * si.nb; })) {
+    stem_status_t st = cuda_status(launch_select(b, hq, hk0 * G, nhk * G, nbtot, nb_max, p->sink_blocks,
+                                                 p->window_blocks, scores,
                                                  budgets, row_ptr, col_idx, stream));
     if (st != STEM_OK) return st;
   }
   return STEM_OK;
 }
 
-stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, const int32_t* row_ptr,
+stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
+                      const int32_t* row_ptr,
                       const int32_t* col_idx, void* out, float* lse, int* status, cudaStream_t stream) {
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
@@ -298,8 +306,10 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.out = out;
   a.lse = lse;
   a.status = status;
+  a.hk0 = hk0;
   // one CTA per CSR row (query head, query block)
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return hq * si.nb; })) {
+  const int G = hq / hkv;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * G * si.nb; })) {
     BsaMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
@@ -343,7 +353,7 @@ stem_status_t stem_score(const stem_qkv_t* qkv, const stem_params_t* params, flo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
   float* vb = vbonus ? vbonus : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_vbonus);
-  return run_score(qkv, params, pl, scores, vb, static_cast<int*>(ws), s);
+  return run_score(qkv, params, pl, 0, qkv->num_kv_heads, scores, vb, static_cast<int*>(ws), s);
 }
 
 stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params, const float* scores,
@@ -356,7 +366,7 @@ stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params, co
   if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
-  return run_select(qkv, params, pl, scores, budgets, row_ptr, col_idx, s);
+  return run_select(qkv, params, pl, 0, qkv->num_kv_heads, true, scores, budgets, row_ptr, col_idx, s);
 }
 
 stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params, const int32_t* row_ptr,
@@ -371,7 +381,7 @@ stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params, c
   if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
-  return run_bsa(qkv, params, pl, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s);
+  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s);
 }
 
 stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, void* out, float* lse,
@@ -393,9 +403,116 @@ stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, v
   int32_t* row_ptr = row_ptr_out ? row_ptr_out : reinterpret_cast<int32_t*>(w + pl.off_rowptr);
   int32_t* col_idx = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(w + pl.off_colidx);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
-  if ((st = run_score(qkv, params, pl, scores, vbonus, status, s)) != STEM_OK) return st;
-  if ((st = run_select(qkv, params, pl, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
-  return run_bsa(qkv, params, pl, row_ptr, col_idx, out, lse, status, s);
+  const int hkv = qkv->num_kv_heads;
+  if ((st = run_score(qkv, params, pl, 0, hkv, scores, vbonus, status, s)) != STEM_OK) return st;
+  if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
+  return run_bsa(qkv, params, pl, 0, hkv, row_ptr, col_idx, out, lse, status, s);
+}
+
+stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_params_t* params, const void* q_host,
+                                const void* k_host, const void* v_host, void* out_dev, float* lse_dev,
+                                void* out_host, float* lse_host, void* ws, size_t ws_bytes, stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if ((st = check_tensors(qkv)) != STEM_OK) return st;
+  if (!q_host || !k_host || !v_host || !out_dev || !lse_dev || !out_host || !lse_host || !ws)
+    return STEM_ERR_INVALID_ARG;
+  if (!aligned16(out_dev)) return STEM_ERR_MISALIGNED;
+  if (ws_bytes < pl.pub.ws_prefill_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  int* status = reinterpret_cast<int*>(w);
+  float* vbonus = reinterpret_cast<float*>(w + pl.off_vbonus);
+  float* scores = reinterpret_cast<float*>(w + pl.off_scores);
+  int32_t* budgets = reinterpret_cast<int32_t*>(w + pl.off_budgets);
+  int32_t* row_ptr = reinterpret_cast<int32_t*>(w + pl.off_rowptr);
+  int32_t* col_idx = reinterpret_cast<int32_t*>(w + pl.off_colidx);
+
+  const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads, G = hq / hkv;
+  const size_t T = static_cast<size_t>(qkv->total_tokens);
+  const size_t elt = qkv->dtype == STEM_FP8_E4M3 ? 1 : 2;
+  const size_t dq = static_cast<size_t>(kHeadDim) * elt;  // bytes of one head row
+  const int ngroups = hkv < 8 ? hkv : 8;
+  const int per = (hkv + ngroups - 1) / ngroups;  // KV heads per group (the last may have fewer)
+
+  // a copy-in and a copy-out stream and the events that chain them with `s`;
+  // released at once: they are freed when the work they order has completed
+  cudaStream_t cin = nullptr, cout = nullptr;
+  cudaEvent_t ev_begin = nullptr, ev_done = nullptr, ev_in[8] = {}, ev_comp[8] = {};
+  auto release = [&]() {
+    if (cin) cudaStreamDestroy(cin);
+    if (cout) cudaStreamDestroy(cout);
+    if (ev_begin) cudaEventDestroy(ev_begin);
+    if (ev_done) cudaEventDestroy(ev_done);
+    for (int g = 0; g < 8; ++g) {
+      if (ev_in[g]) cudaEventDestroy(ev_in[g]);
+      if (ev_comp[g]) cudaEventDestroy(ev_comp[g]);
+    }
+  };
+  auto fail = [&](cudaError_t e) {
+    release();
+    return cuda_status(e);
+  };
+  cudaError_t e = cudaStreamCreateWithFlags(&cin, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&cout, cudaStreamNonBlocking);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_begin, cudaEventDisableTiming);
+  if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_done, cudaEventDisableTiming);
+  for (int g = 0; g < ngroups && e == cudaSuccess; ++g) {
+    e = cudaEventCreateWithFlags(&ev_in[g], cudaEventDisableTiming);
+    if (e == cudaSuccess) e = cudaEventCreateWithFlags(&ev_comp[g], cudaEventDisableTiming);
+  }
+  if (e != cudaSuccess) return fail(e);
+
+  // inputs: one 2-d copy per tensor and group (the group's heads are a slab of
+  // every token row)
+  if ((e = cudaEventRecord(ev_begin, s)) != cudaSuccess || (e = cudaStreamWaitEvent(cin, ev_begin, 0)) != cudaSuccess)
+    return fail(e);
+  for (int g = 0; g < ngroups; ++g) {
+    const int hk0 = g * per, nhk = (hk0 + per <= hkv) ? per : hkv - hk0;
+    if (nhk <= 0) break;
+    const size_t oq = static_cast<size_t>(hk0) * G * dq, ok = static_cast<size_t>(hk0) * dq;
+    e = cudaMemcpy2DAsync(static_cast<uint8_t*>(const_cast<void*>(qkv->q)) + oq, hq * dq, static_cast<const uint8_t*>(q_host) + oq,
+                          hq * dq, nhk * G * dq, T, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<uint8_t*>(const_cast<void*>(qkv->k)) + ok, hkv * dq, static_cast<const uint8_t*>(k_host) + ok,
+                            hkv * dq, nhk * dq, T, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<uint8_t*>(const_cast<void*>(qkv->v)) + ok, hkv * dq, static_cast<const uint8_t*>(v_host) + ok,
+                            hkv * dq, nhk * dq, T, cudaMemcpyHostToDevice, cin);
+    if (e == cudaSuccess) e = cudaEventRecord(ev_in[g], cin);
+    if (e != cudaSuccess) return fail(e);
+  }
+  // compute on `s`, group by group; results back on the copy-out stream
+  if ((st = clear_status(ws, s)) != STEM_OK) {
+    release();
+    return st;
+  }
+  for (int g = 0; g < ngroups; ++g) {
+    const int hk0 = g * per, nhk = (hk0 + per <= hkv) ? per : hkv - hk0;
+    if (nhk <= 0) break;
+    if ((e = cudaStreamWaitEvent(s, ev_in[g], 0)) != cudaSuccess) return fail(e);
+    if ((st = run_score(qkv, params, pl, hk0, nhk, scores, vbonus, status, s)) != STEM_OK ||
+        (st = run_select(qkv, params, pl, hk0, nhk, g == 0, scores, budgets, row_ptr, col_idx, s)) != STEM_OK ||
+        (st = run_bsa(qkv, params, pl, hk0, nhk, row_ptr, col_idx, out_dev, lse_dev, status, s)) != STEM_OK) {
+      release();
+      return st;
+    }
+    if ((e = cudaEventRecord(ev_comp[g], s)) != cudaSuccess || (e = cudaStreamWaitEvent(cout, ev_comp[g], 0)) != cudaSuccess)
+      return fail(e);
+    const size_t oo = static_cast<size_t>(hk0) * G * kHeadDim * 2;  // O is bf16
+    e = cudaMemcpy2DAsync(static_cast<uint8_t*>(out_host) + oo, hq * kHeadDim * 2,
+                          static_cast<const uint8_t*>(out_dev) + oo, hq * kHeadDim * 2, nhk * G * kHeadDim * 2, T,
+                          cudaMemcpyDeviceToHost, cout);
+    if (e == cudaSuccess)
+      e = cudaMemcpyAsync(lse_host + static_cast<size_t>(hk0) * G * T, lse_dev + static_cast<size_t>(hk0) * G * T,
+                          static_cast<size_t>(nhk) * G * T * sizeof(float), cudaMemcpyDeviceToHost, cout);
+    if (e != cudaSuccess) return fail(e);
+  }
+  if ((e = cudaEventRecord(ev_done, cout)) != cudaSuccess || (e = cudaStreamWaitEvent(s, ev_done, 0)) != cudaSuccess)
+    return fail(e);
+  release();
+  return STEM_OK;
 }
 
 stem_status_t stem_read_device_status(const void* ws, stem_stream_t stream, stem_status_t* out) {

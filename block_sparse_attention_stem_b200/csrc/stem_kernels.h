@@ -30,6 +30,7 @@ struct BsaMaps {
 
 struct ScoreArgs {
   int hq, hkv, nbtot, nb_max, stride;
+  int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
   float scale;              // 1 / (sqrt(d) s n)
   const float* q_scale;     // fp8 only
   const float* k_scale;
@@ -40,6 +41,7 @@ struct ScoreArgs {
 
 struct BsaArgs {
   int hq, hkv, nbtot, total_tokens;
+  int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
   float scale_log2;         // softmax scale * log2(e)
   const float* q_scale;     // fp8 only
   const float* k_scale;
@@ -52,13 +54,15 @@ struct BsaArgs {
   int* status;
 };
 
-cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int nbtot,
-                         float beta, float* vbonus, cudaStream_t stream);
+// KV heads hk0 .. hk0 + nhk - 1 only
+cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
+                         int nhk, int nbtot, float beta, float* vbonus, cudaStream_t stream);
 cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args, bool fp8,
                          cudaStream_t stream);
 cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_per_head, double rho, double mu,
                           int sink, int window, int mode, int32_t* budgets, int32_t* row_ptr, cudaStream_t stream);
-cudaError_t launch_select(const SeqBatch& batch, int hq, int nbtot, int nb_max, int sink, int window,
+// rows of query heads h0 .. h0 + nh - 1 only (batch items: nh * nb per sequence)
+cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int nbtot, int nb_max, int sink, int window,
                           const float* scores, const int32_t* budgets, const int32_t* row_ptr, int32_t* col_idx,
                           cudaStream_t stream);
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,

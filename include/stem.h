@@ -171,8 +171,8 @@ STEM_API stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* p
  *   sigma = softmax_scale (or 1/sqrt(d)), times q_scale*k_scale for fp8.
  * out bf16 [T, Hq, d]; lse fp32 [Hq][T].  Lists must be strictly ascending with
  * 0 <= j <= i; a violating entry is skipped and STEM_ERR_BAD_BLOCKLIST recorded.
- * An empty row gives out = 0 and lse = -inf.  fp8: P is rounded to e4m3 for the
- * P.V product. */
+ * An empty row gives out = 0 and lse = -inf.  fp8: P*224 is split into two e4m3
+ * terms (hi + lo) whose two P.V products accumulate into O. */
 STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params,
                            const int32_t* row_ptr, const int32_t* col_idx,
                            void* out, float* lse,
@@ -185,6 +185,28 @@ STEM_API stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* 
                            void* out, float* lse,
                            int32_t* row_ptr_out, int32_t* col_idx_out,
                            void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* stem_prefill for inputs and outputs in host memory, with the transfers
+ * overlapped with the computation.
+ *   qkv        describes the layer as for stem_prefill; qkv->q, k, v point to
+ *              DEVICE buffers of the full [T, H, d] size, which this call fills.
+ *   q_host, k_host, v_host  the inputs in host memory, same layout (page-locked
+ *              memory is needed for the copies to run asynchronously).
+ *   out_dev, lse_dev        device buffers for O and LSE (as stem_prefill's).
+ *   out_host, lse_host      host destinations for O bf16 [T, Hq, d] and LSE
+ *              fp32 [Hq][T].
+ *   ws, ws_bytes            as stem_prefill (ws_bytes >= plan.ws_prefill_bytes).
+ * The layer is processed one group of KV heads (with their query heads) at a
+ * time, at most 8 groups: the inputs of group g+1 are copied while group g
+ * computes, the results of group g are copied back while g+1 computes.  The
+ * work is ordered after the work already on `stream`, and `stream` completes
+ * only once the results are in host memory; the call itself only enqueues.
+ * Results equal stem_prefill's bit for bit.  Host-side errors as stem_prefill;
+ * STEM_ERR_INVALID_ARG also for a NULL host pointer. */
+STEM_API stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_params_t* params,
+                                const void* q_host, const void* k_host, const void* v_host,
+                                void* out_dev, float* lse_dev, void* out_host, float* lse_host,
+                                void* ws, size_t ws_bytes, stem_stream_t stream);
 
 /* stem_prefill without a caller workspace, for callers that cannot allocate
  * device memory (code running where cudaMalloc is not allowed or not wanted:
