@@ -71,6 +71,10 @@ import numpy as np
 RELATIVE = 0
 ABSOLUTE = 1
 
+# value-magnitude bonus forms (see value_bonus)
+BONUS_LOG = 0           # beta * max(0, ln ||v||^2)
+BONUS_STANDARDIZED = 1  # beta * ReLU(z-score of ln ||v||^2)
+
 
 @dataclass
 class Params:
@@ -85,6 +89,7 @@ class Params:
     window_blocks: int = 4
     softmax_scale: float = 0.0  # 0 -> 1/sqrt(head_dim)
     budget_mode: int = RELATIVE
+    bonus_mode: int = BONUS_LOG
 
 
 # --------------------------------------------------------------------------
@@ -156,19 +161,47 @@ def seq_blocks(cu_seqlens, block: int = 128):
 # the same).
 # --------------------------------------------------------------------------
 
-def value_bonus(v: np.ndarray, cu_seqlens, beta: float, block: int = 128) -> np.ndarray:
-    """v: fp64 [T, Hkv, d].  Returns bonus fp64 [Hkv, NBtot]."""
+def value_bonus(v: np.ndarray, cu_seqlens, beta: float, block: int = 128, mode: int = BONUS_LOG) -> np.ndarray:
+    """v: fp64 [T, Hkv, d].  Returns bonus fp64 [Hkv, NBtot].
+
+    x_j = ln max_{t in block j} ||v_t||^2 (gist-zh §2.2; the max is pooled
+    over the block's tokens before the log, which is the same as pooling the
+    logs).
+
+    mode BONUS_LOG (gist-zh §2.2, gist-de §2 C): bonus_j = beta * max(0, x_j);
+    ln 0 = -inf gives 0.
+
+    mode BONUS_STANDARDIZED (AngelSlim doc §2.1 and the Stem overview's OAM
+    formula: lambda * ReLU(v_bar_j), v_bar the standardized log value norm):
+    v_bar_j = (x_j - mean) / std over the finite x of the same sequence and KV
+    head (all its key blocks; population std); bonus_j = beta * max(0, v_bar_j).
+    A block whose x is not finite gets 0, and so does every block when the std
+    is 0 or fewer than one finite x exists.  The pages do not define the
+    statistics' scope; this is the reading used here."""
     seqs, nbtot = seq_blocks(cu_seqlens, block)
     hkv = v.shape[1]
     bonus = np.zeros((hkv, nbtot), dtype=np.float64)
     for (o, L, nb, g0) in seqs:
+        x = np.empty((hkv, nb), dtype=np.float64)
         for j in range(nb):
             rows = v[o + j * block: o + min((j + 1) * block, L)]  # [n, Hkv, d]
             sq = np.sum(rows * rows, axis=2)  # ||v_t||^2  [n, Hkv]
             m = np.max(sq, axis=0)  # max over the tokens of block j
             with np.errstate(divide="ignore"):
-                lg = np.log(m)  # ln 0 = -inf -> bonus 0
-            bonus[:, g0 + j] = beta * np.maximum(0.0, lg)
+                x[:, j] = np.log(m)  # ln 0 = -inf
+        if mode == BONUS_LOG:
+            bonus[:, g0:g0 + nb] = beta * np.maximum(0.0, x)
+            continue
+        for h in range(hkv):
+            fin = np.isfinite(x[h])
+            if not fin.any():
+                continue
+            mean = x[h][fin].mean()
+            std = math.sqrt(((x[h][fin] - mean) ** 2).mean())
+            if std == 0.0:
+                continue
+            z = np.where(fin, (np.where(fin, x[h], 0.0) - mean) / std, -np.inf)
+            bonus[h, g0:g0 + nb] = beta * np.maximum(0.0, z)
     return bonus
 
 
@@ -260,7 +293,7 @@ def block_scores(q: np.ndarray, k: np.ndarray, v: np.ndarray, cu_seqlens, p: Par
     nb_max = max(nb for (_, _, nb, _) in seqs)
     hq, hkv = q.shape[1], k.shape[1]
     G = hq // hkv
-    bonus = value_bonus(v, cu_seqlens, p.beta, B)
+    bonus = value_bonus(v, cu_seqlens, p.beta, B, p.bonus_mode)
     S = np.full((hq, nbtot, nb_max), -np.inf, dtype=np.float64)
     chunk_blocks = max(1, p.chunk_size // B)
     for (o, L, nb, g0) in seqs:
@@ -291,7 +324,9 @@ def block_score_row(q: np.ndarray, k: np.ndarray, v: np.ndarray, i: int, p: Para
     ng_valid = cdiv(L, s)
     a0, a1 = i * gpb, min((i + 1) * gpb, ng_valid)
     D = downsampled_scores(q, k, s, p.norm, groups=(a0, a1), key_groups=min((i + 1) * gpb, ng_valid))[0]
-    bonus = value_bonus(v[:min((i + 1) * B, L)], [0, min((i + 1) * B, L)], p.beta, B)[0]
+    # the standardized form needs every block of the sequence; the log form
+    # only blocks 0..i, so both take the whole sequence here
+    bonus = value_bonus(v, [0, L], p.beta, B, p.bonus_mode)[0]
     out = np.empty(i + 1)
     for j in range(i + 1):
         out[j] = D[:, j * gpb:min((j + 1) * gpb, ng_valid)].max() + bonus[j]

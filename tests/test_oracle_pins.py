@@ -259,6 +259,52 @@ def test_value_bonus_special_cases():
     assert b[0].tolist() == pytest.approx([0.4, 0.0, 0.0], abs=1e-15)
 
 
+def _blocks_with_norms(sq_norms, block=16, d=4):
+    """V [len(sq_norms) * block, 1, d] whose block j has max ||v_t||^2 = sq_norms[j]
+    (one token at that norm, the others smaller)."""
+    v = np.zeros((len(sq_norms) * block, 1, d))
+    for j, n2 in enumerate(sq_norms):
+        v[j * block, 0, 0] = math.sqrt(n2)
+        v[j * block + 1: (j + 1) * block, 0, 1] = 0.5 * math.sqrt(n2)
+    return v
+
+
+def test_standardized_bonus_closed_forms():
+    """Standardized OAM (AngelSlim doc §2.1: lambda ReLU(v_bar_j)): x_j = ln of
+    the block's largest squared norm, z-scored over the sequence's blocks.
+    Two blocks: z = -1, +1.  Three equally spaced x: z = -sqrt(3/2), 0, +sqrt(3/2)."""
+    beta = 0.3
+    b2 = O.value_bonus(_blocks_with_norms([math.exp(0.7), math.exp(5.0)]), [0, 32], beta, 16, O.BONUS_STANDARDIZED)
+    assert b2[0].tolist() == pytest.approx([0.0, beta], abs=1e-12)
+    b3 = O.value_bonus(_blocks_with_norms([1.0, math.e, math.e ** 2]), [0, 48], beta, 16, O.BONUS_STANDARDIZED)
+    assert b3[0].tolist() == pytest.approx([0.0, 0.0, beta * math.sqrt(1.5)], abs=1e-12)
+    # the log form on the same input: beta * max(0, x)
+    b3l = O.value_bonus(_blocks_with_norms([1.0, math.e, math.e ** 2]), [0, 48], beta, 16, O.BONUS_LOG)
+    assert b3l[0].tolist() == pytest.approx([0.0, beta, 2 * beta], abs=1e-12)
+
+
+def test_standardized_bonus_is_scale_invariant_and_handles_degenerate_blocks():
+    rng = np.random.default_rng(21)
+    v = rng.standard_normal((5 * 16, 2, 4)) * np.exp(rng.standard_normal((5 * 16, 2, 1)))
+    b = O.value_bonus(v, [0, 80], 0.2, 16, O.BONUS_STANDARDIZED)
+    # scaling V scales every ||v||^2 by c^2: x shifts, z does not
+    assert np.allclose(O.value_bonus(7.5 * v, [0, 80], 0.2, 16, O.BONUS_STANDARDIZED), b, rtol=0, atol=1e-12)
+    assert not np.allclose(O.value_bonus(7.5 * v, [0, 80], 0.2, 16, O.BONUS_LOG),
+                           O.value_bonus(v, [0, 80], 0.2, 16, O.BONUS_LOG))
+    # z-scores of a head sum to zero: the bonus is the positive part, times beta
+    x = np.array([[np.log(np.max(np.sum(v[j * 16:(j + 1) * 16, h] ** 2, axis=1))) for j in range(5)] for h in range(2)])
+    z = (x - x.mean(axis=1, keepdims=True)) / x.std(axis=1, keepdims=True)
+    assert np.allclose(b, 0.2 * np.maximum(0, z), atol=1e-12)
+    # equal norms: std 0 -> no bonus; a zero block is left out of the statistics
+    assert not O.value_bonus(_blocks_with_norms([2.0, 2.0, 2.0]), [0, 48], 0.2, 16, O.BONUS_STANDARDIZED).any()
+    vz = _blocks_with_norms([1.0, 0.0, math.e ** 2])
+    bz = O.value_bonus(vz, [0, 48], 0.5, 16, O.BONUS_STANDARDIZED)
+    assert bz[0].tolist() == pytest.approx([0.0, 0.0, 0.5], abs=1e-12)  # z over {0, 2}: -1, +1
+    # statistics are per sequence: a second sequence does not change the first one's bonus
+    two = np.concatenate([vz, _blocks_with_norms([100.0, 1e-3])])
+    assert O.value_bonus(two, [0, 48, 80], 0.5, 16, O.BONUS_STANDARDIZED)[0, :3].tolist() == bz[0].tolist()
+
+
 def test_oam_log_form_ranks_like_product_form():
     """HPC-BSA article §2.2: the log turns the product exp(routing) * magnitude
     into a sum without changing the ranking.  Top-k by the additive score must
@@ -379,13 +425,14 @@ def test_skipped_block_changes_only_its_rows_weights():
     np.testing.assert_allclose(np.exp(l2[0, t]), lf - lbk, rtol=1e-12)
 
 
-def test_single_row_scoring_equals_full_matrix_row():
+@pytest.mark.parametrize("bonus_mode", [O.BONUS_LOG, O.BONUS_STANDARDIZED])
+def test_single_row_scoring_equals_full_matrix_row(bonus_mode):
     rng = np.random.default_rng(21)
     B, s, d, L = 32, 8, 8, 5 * 32 + 9
     q = rng.standard_normal((L, 4, d))
     k = rng.standard_normal((L, 2, d))
-    v = rng.standard_normal((L, 2, d)) * 3
-    p = O.Params(block_size=B, stride=s, chunk_size=64, beta=0.3, norm=1.3)
+    v = rng.standard_normal((L, 2, d)) * 3 * np.exp(rng.standard_normal((L, 2, 1)))
+    p = O.Params(block_size=B, stride=s, chunk_size=64, beta=0.3, norm=1.3, bonus_mode=bonus_mode)
     full = O.block_scores(q, k, v, [0, L], p)
     for h in range(4):
         for i in range(6):
