@@ -54,8 +54,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
-    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack"], default="default",
-                    help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack")
+    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality"], default="default",
+                    help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack; "
+                         "quality: reconstruction error against dense attention (32K)")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
     return ap.parse_args(argv)
 
@@ -556,6 +557,64 @@ def run_sweep(args):
     print(json.dumps(res), flush=True)
 
 
+def run_quality(args):
+    """How much of dense attention the selected blocks reproduce, on the 32K
+    workload: relative Frobenius error of O against dense attention (the same
+    kernel over every causal block) and the softmax mass the selection keeps,
+    mean over rows of exp(lse_sparse - lse_dense).  Compares the output-aware
+    metric (beta = 0.2) with the routing score alone (beta = 0), and the
+    position-decay budget (mu = 0.7) with a uniform one (mu = 1) at the same
+    kept-block count.  Synthetic inputs: a check of the method's direction, not
+    an accuracy benchmark."""
+    import torch
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+    w0 = I.workload("qwen32k")
+    inp = I.make_inputs(w0, device="cuda")
+    cu = w0.cu_seqlens()
+    qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], cu, cu_seqlens_dev=inp["cu_seqlens"])
+    nb = math.ceil(w0.seqlens[0] / 128)
+    hq = w0.num_q_heads
+    # dense reference: every causal block listed
+    counts = torch.arange(1, nb + 1, dtype=torch.int64).repeat(hq)
+    drp = torch.zeros(hq * nb + 1, dtype=torch.int32)
+    drp[1:] = torch.cumsum(counts, 0).to(torch.int32)
+    dci = torch.cat([torch.arange(c, dtype=torch.int32) for c in range(1, nb + 1)]).repeat(hq)
+    params0 = b.make_params(**w0.params())
+    o_dense, l_dense, _ = b.stem_bsa_fwd(qkv, params0, drp.cuda(), dci.cuda())
+    o_dense = o_dense.float()
+    nrm = torch.linalg.vector_norm(o_dense).item()
+
+    def nnz_of(**kw):
+        return b.stem_plan(qkv, b.make_params(**dict(w0.params(), **kw))).nnz_per_head
+
+    target = nnz_of(mu=0.7, keep_ratio=w0.keep_ratio)
+    lo, hi = 0.01, 1.0  # uniform-budget keep ratio with the same kept-block count
+    for _ in range(40):
+        mid = 0.5 * (lo + hi)
+        lo, hi = (mid, hi) if nnz_of(mu=1.0, keep_ratio=mid) < target else (lo, mid)
+    rho_eq = hi
+    causal = nb * (nb + 1) // 2
+    points = []
+    for label, kw in (("stem: OAM beta 0.2, TPD mu 0.7", dict(beta=0.2, mu=0.7)),
+                      ("routing score only: beta 0, mu 0.7", dict(beta=0.0, mu=0.7)),
+                      ("OAM beta 0.2, uniform budget mu 1 (same kept blocks)", dict(beta=0.2, mu=1.0, keep_ratio=rho_eq)),
+                      ("routing score only, uniform budget", dict(beta=0.0, mu=1.0, keep_ratio=rho_eq))):
+        params = b.make_params(**dict(w0.params(), **kw))
+        out, lse, _, _, ws = b.stem_prefill(qkv, params, return_lists=False)
+        torch.cuda.synchronize()
+        assert b.stem_read_device_status(ws) == 0
+        err = torch.linalg.vector_norm(out.float() - o_dense).item() / nrm
+        mass = torch.exp(lse - l_dense).mean().item()
+        pl = b.stem_plan(qkv, params)
+        points.append(dict(selection=label, density=round(pl.nnz_per_head / causal, 4),
+                           rel_error_vs_dense=round(err, 5), softmax_mass_kept=round(mass, 5), **kw))
+    res = {"metric": "attention reconstruction vs dense (32K, synthetic)", "unit": "relative Frobenius error",
+           "higher_is_better": False, "points": points, "config": describe(w0), "dtype": "bf16",
+           "data": "synthetic (seeded, device RNG)"}
+    print(json.dumps(res), flush=True)
+
+
 def run_fp8stack(args):
     """The fp8 varlen stack: 4 packed sequences {8192, 16384, 40960, 98304},
     e4m3 inputs with per-head scales, one independently seeded layer per step
@@ -595,6 +654,8 @@ def main(argv=None):
         run_reference(args)
     elif args.mode == "sweep":
         run_sweep(args)
+    elif args.mode == "quality":
+        run_quality(args)
     elif args.mode == "fp8stack":
         run_fp8stack(args)
     else:

@@ -18,7 +18,8 @@ namespace stem {
 template <bool kFp8>
 __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const uint8_t* __restrict__ v,
                                                     const float* __restrict__ v_scale, int hkv, int hk0, int nhk,
-                                                    int nbtot, float beta, float* __restrict__ vbonus) {
+                                                    int nbtot, float beta, bool raw_log,
+                                                    float* __restrict__ vbonus) {
   extern __shared__ unsigned int s_max[];  // [nhk] bit patterns of non-negative floats (KV heads hk0 ..)
   const int s = find_seq(batch, blockIdx.x);
   const int j = blockIdx.x - batch.item0[s];
@@ -77,21 +78,89 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
   for (int h = threadIdx.x; h < nhk; h += blockDim.x) {
     const float m = __uint_as_float(s_max[h]);
     const float lg = logf(m);  // ln 0 = -inf -> bonus 0
-    vbonus[static_cast<size_t>(hk0 + h) * nbtot + g] = beta * fmaxf(0.f, lg);
+    vbonus[static_cast<size_t>(hk0 + h) * nbtot + g] = raw_log ? lg : beta * fmaxf(0.f, lg);
   }
 }
 
 cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
-                         int nhk, int nbtot, float beta, float* vbonus, cudaStream_t stream) {
+                         int nhk, int nbtot, float beta, bool raw_log, float* vbonus, cudaStream_t stream) {
   const int items = batch.item0[batch.n];
   if (items == 0 || nhk <= 0) return cudaSuccess;
   const size_t smem = sizeof(unsigned int) * static_cast<size_t>(nhk);
   if (fp8)
     vnorm_kernel<true><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                     nbtot, beta, vbonus);
+                                                     nbtot, beta, raw_log, vbonus);
   else
     vnorm_kernel<false><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                      nbtot, beta, vbonus);
+                                                      nbtot, beta, raw_log, vbonus);
+  return cudaGetLastError();
+}
+
+// One CTA per (sequence, KV head): mean and population std of the finite
+// x = ln max ||v||^2 over the sequence's blocks (two passes, fp64 sums), then
+// bonus = beta * max(0, (x - mean) / std); 0 for a non-finite x, and for every
+// block when std = 0 or no x is finite.  AngelSlim doc §2.1 (lambda *
+// ReLU(v_bar), v_bar the standardized log value norm).
+__global__ void __launch_bounds__(256) bonus_standardize_kernel(const SeqBatch batch, int hk0, int nbtot,
+                                                                float beta, float* __restrict__ vbonus) {
+  __shared__ double s_red[2][8];
+  const int s = find_seq(batch, blockIdx.x);
+  const int hk = hk0 + (blockIdx.x - batch.item0[s]);
+  const int nb = batch.nb[s];
+  float* x = vbonus + static_cast<size_t>(hk) * nbtot + batch.g0[s];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  // block-wide sum of (a, b) over the threads
+  auto reduce2 = [&](double a, double b, double* ra, double* rb) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      a += __shfl_xor_sync(0xffffffffu, a, off);
+      b += __shfl_xor_sync(0xffffffffu, b, off);
+    }
+    if (lane == 0) {
+      s_red[0][w] = a;
+      s_red[1][w] = b;
+    }
+    __syncthreads();
+    double ta = 0.0, tb = 0.0;
+    for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) {
+      ta += s_red[0][i];
+      tb += s_red[1][i];
+    }
+    __syncthreads();
+    *ra = ta;
+    *rb = tb;
+  };
+  double sum = 0.0, cnt = 0.0;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const float v = x[j];
+    if (isfinite(v)) {
+      sum += v;
+      cnt += 1.0;
+    }
+  }
+  double tsum, tcnt;
+  reduce2(sum, cnt, &tsum, &tcnt);
+  const double mean = tcnt > 0.0 ? tsum / tcnt : 0.0;
+  double sq = 0.0, unused = 0.0;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const float v = x[j];
+    if (isfinite(v)) sq += (v - mean) * (v - mean);
+  }
+  double tsq, tun;
+  reduce2(sq, unused, &tsq, &tun);
+  const double sd = tcnt > 0.0 ? sqrt(tsq / tcnt) : 0.0;
+  for (int j = threadIdx.x; j < nb; j += blockDim.x) {
+    const float v = x[j];
+    const double z = (sd > 0.0 && isfinite(v)) ? (v - mean) / sd : 0.0;
+    x[j] = beta * static_cast<float>(z > 0.0 ? z : 0.0);
+  }
+}
+
+cudaError_t launch_bonus_standardize(const SeqBatch& batch, int hk0, int nbtot, float beta, float* vbonus,
+                                     cudaStream_t stream) {
+  const int items = batch.item0[batch.n];
+  if (items == 0) return cudaSuccess;
+  bonus_standardize_kernel<<<items, 256, 0, stream>>>(batch, hk0, nbtot, beta, vbonus);
   return cudaGetLastError();
 }
 

@@ -59,6 +59,7 @@ stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
   if (p->sink_blocks < 0 || p->window_blocks < 1) return STEM_ERR_INVALID_ARG;
   if (!(p->softmax_scale >= 0.0) || !std::isfinite(p->softmax_scale)) return STEM_ERR_INVALID_ARG;
   if (p->budget_mode != STEM_BUDGET_RELATIVE && p->budget_mode != STEM_BUDGET_ABSOLUTE) return STEM_ERR_INVALID_ARG;
+  if (p->bonus_mode != STEM_BONUS_LOG && p->bonus_mode != STEM_BONUS_STANDARDIZED) return STEM_ERR_INVALID_ARG;
   return STEM_OK;
 }
 
@@ -228,7 +229,14 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
   for (const SeqBatch& b : make_batches(pl, [](const SeqInfo& si) { return si.nb; })) {
     stem_status_t st = cuda_status(
-        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, hk0, nhk, nbtot, static_cast<float>(p->beta), vbonus, stream));
+        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, hk0, nhk, nbtot, static_cast<float>(p->beta),
+                     p->bonus_mode == STEM_BONUS_STANDARDIZED, vbonus, stream));
+    if (st != STEM_OK) return st;
+  }
+  // standardized bonus: z-score over each sequence's blocks, per KV head
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo&) { return nhk; })) {
+    if (p->bonus_mode != STEM_BONUS_STANDARDIZED) break;
+    stem_status_t st = cuda_status(launch_bonus_standardize(b, hk0, nbtot, static_cast<float>(p->beta), vbonus, stream));
     if (st != STEM_OK) return st;
   }
   ScoreArgs a{};

@@ -54,9 +54,14 @@ struct BsaArgs {
   int* status;
 };
 
-// KV heads hk0 .. hk0 + nhk - 1 only
+// KV heads hk0 .. hk0 + nhk - 1 only.  raw_log: write x = ln max ||v||^2 for a
+// later launch_bonus_standardize instead of beta * max(0, x).
 cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
-                         int nhk, int nbtot, float beta, float* vbonus, cudaStream_t stream);
+                         int nhk, int nbtot, float beta, bool raw_log, float* vbonus, cudaStream_t stream);
+// vbonus[hk][g] = beta * max(0, (x - mean) / std) over the finite x of each
+// sequence, for KV heads hk0 .. hk0 + (items per sequence) - 1.
+cudaError_t launch_bonus_standardize(const SeqBatch& batch, int hk0, int nbtot, float beta, float* vbonus,
+                                     cudaStream_t stream);
 cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args, bool fp8,
                          cudaStream_t stream);
 cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_per_head, double rho, double mu,

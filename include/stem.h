@@ -77,6 +77,13 @@ typedef enum { STEM_BF16 = 0, STEM_FP8_E4M3 = 1 } stem_dtype_t;
  *   ABSOLUTE: k_start = ceil(rho * NB_s) for every row of the sequence. */
 typedef enum { STEM_BUDGET_RELATIVE = 0, STEM_BUDGET_ABSOLUTE = 1 } stem_budget_mode_t;
 
+/* Form of the value-magnitude bonus of the output-aware metric. */
+typedef enum {
+  STEM_BONUS_LOG = 0,          /* beta * max(0, ln ||v||^2)  [gist-zh §2.2; gist-de §2 C] */
+  STEM_BONUS_STANDARDIZED = 1  /* beta * ReLU(standardized ln ||v||^2)  [AngelSlim doc §2.1;
+                                  the statistics' scope is this library's reading] */
+} stem_bonus_mode_t;
+
 /* Method parameters (AngelSlim documentation §6 defaults in brackets). */
 typedef struct {
   int32_t block_size;     /* attention block [128]; only 128 is supported */
@@ -90,6 +97,7 @@ typedef struct {
   int32_t window_blocks;  /* trailing causal blocks always kept, the diagonal included [4]; >= 1 */
   double  softmax_scale;  /* attention logit scale; 0 selects 1/sqrt(head_dim) */
   int32_t budget_mode;    /* stem_budget_mode_t */
+  int32_t bonus_mode;     /* stem_bonus_mode_t [STEM_BONUS_LOG] */
 } stem_params_t;
 
 /* Query/key/value description shared by all calls. */
@@ -136,7 +144,11 @@ STEM_API stem_status_t stem_plan(const stem_qkv_t* qkv, const stem_params_t* par
 
 /* Block scores [AngelSlim doc §2.1; gist-zh §2.2 OAM and §2.3 anti-diagonal
  * downsampling; gist-de §2 C].
- *   vbonus[hk][g] = beta * max(0, ln max_{t in block g} ||v_t||^2)
+ *   x[hk][g]      = ln max_{t in block g} ||v_t||^2
+ *   vbonus[hk][g] = beta * max(0, x)                       (STEM_BONUS_LOG)
+ *                   beta * max(0, (x - mean) / std)        (STEM_BONUS_STANDARDIZED:
+ *                   mean and population std of the finite x of the same sequence
+ *                   and KV head; 0 where x is not finite or std = 0)
  *   D[h][a][b]    = sum_{u<s} q[a s + u, h] . k[b s + s-1-u, h/G] / (sqrt(d) s n)
  *   scores[h][g][j] = max over the query groups a of block g and key groups b of
  *                     block j of D + vbonus[h/G][g0+j]   for j <= i (local index);
