@@ -71,6 +71,10 @@ import numpy as np
 RELATIVE = 0
 ABSOLUTE = 1
 
+# block-list granularity under GQA (see select)
+LIST_PER_HEAD = 0   # every query head selects its own blocks
+LIST_PER_GROUP = 1  # one list per KV head, from the max over its query heads
+
 # value-magnitude bonus forms (see value_bonus)
 BONUS_LOG = 0           # beta * max(0, ln ||v||^2)
 BONUS_STANDARDIZED = 1  # beta * ReLU(z-score of ln ||v||^2)
@@ -90,6 +94,7 @@ class Params:
     softmax_scale: float = 0.0  # 0 -> 1/sqrt(head_dim)
     budget_mode: int = RELATIVE
     bonus_mode: int = BONUS_LOG
+    list_mode: int = LIST_PER_HEAD
 
 
 # --------------------------------------------------------------------------
@@ -400,9 +405,28 @@ def select_row(scores_row: np.ndarray, i: int, b: int, sink: int, window: int) -
     return sorted(F + take)
 
 
-def select(scores: np.ndarray, cu_seqlens, p: Params):
+def group_pooled_scores(scores: np.ndarray, hkv: int) -> np.ndarray:
+    """GQA-shared lists (NEXT variant of the selection; HPC-BSA article §3.1
+    block lists shared by the query heads of a KV head): every query head's
+    score row becomes the elementwise max over the query heads of its KV
+    group, NaN counted as -inf (the selection's NaN rule)."""
+    hq = scores.shape[0]
+    G = hq // hkv
+    out = np.empty_like(scores)
+    for hk in range(hkv):
+        grp = scores[hk * G:(hk + 1) * G]
+        pooled = np.where(np.isnan(grp), -np.inf, grp).max(axis=0)
+        out[hk * G:(hk + 1) * G] = pooled
+    return out
+
+
+def select(scores: np.ndarray, cu_seqlens, p: Params, hkv: int | None = None):
     """scores fp64 [Hq, NBtot, nb_max] -> (budgets [Hq*NBtot], row_ptr
-    [Hq*NBtot+1], col_idx [nnz]) with CSR row r = h*NBtot + g."""
+    [Hq*NBtot+1], col_idx [nnz]) with CSR row r = h*NBtot + g.  With
+    p.list_mode == LIST_PER_GROUP (hkv required) the query heads of a KV
+    group select on their pooled scores and so share one list."""
+    if p.list_mode == LIST_PER_GROUP:
+        scores = group_pooled_scores(scores, hkv)
     seqs, nbtot = seq_blocks(cu_seqlens, p.block_size)
     hq = scores.shape[0]
     bud = budgets(cu_seqlens, p)
@@ -512,7 +536,7 @@ def full_csr(cu_seqlens, hq: int, block: int = 128):
 def prefill(q, k, v, cu_seqlens, p: Params):
     """score -> select -> block-sparse attention, all in fp64."""
     S = block_scores(q, k, v, cu_seqlens, p)
-    bud, row_ptr, col_idx = select(S, cu_seqlens, p)
+    bud, row_ptr, col_idx = select(S, cu_seqlens, p, hkv=k.shape[1])
     O, LSE = bsa(q, k, v, cu_seqlens, row_ptr, col_idx, p)
     return dict(scores=S, budgets=bud, row_ptr=row_ptr, col_idx=col_idx, out=O, lse=LSE)
 

@@ -305,6 +305,67 @@ def test_standardized_bonus_is_scale_invariant_and_handles_degenerate_blocks():
     assert O.value_bonus(two, [0, 48, 80], 0.5, 16, O.BONUS_STANDARDIZED)[0, :3].tolist() == bz[0].tolist()
 
 
+def _rows(rp, ci):
+    return [ci[rp[r]:rp[r + 1]].tolist() for r in range(len(rp) - 1)]
+
+
+def test_group_lists_pool_by_max_and_are_shared():
+    """GQA-shared lists: for every (KV head, query block) the G query heads get
+    one list, the per-head selection applied to the elementwise max of their
+    score rows (checked against loops over the heads, not the vectorised max)."""
+    rng = np.random.default_rng(31)
+    hq, hkv, nb = 6, 2, 9
+    cu = [0, nb * 16]
+    p = O.Params(block_size=16, keep_ratio=0.4, mu=0.8, sink_blocks=1, window_blocks=1, list_mode=O.LIST_PER_GROUP)
+    sc = np.full((hq, nb, nb), -np.inf)
+    for h in range(hq):
+        for i in range(nb):
+            sc[h, i, :i + 1] = rng.standard_normal(i + 1)
+    sc[4, 3, 1] = np.nan  # NaN counts as -inf in the pooling too
+    bud, rp, ci = O.select(sc, cu, p, hkv=hkv)
+    rows = _rows(rp, ci)
+    G = hq // hkv
+    for hk in range(hkv):
+        for i in range(nb):
+            pooled = []
+            for j in range(i + 1):
+                best = -math.inf
+                for h in range(hk * G, (hk + 1) * G):
+                    x = sc[h, i, j]
+                    if not math.isnan(x) and x > best:
+                        best = x
+                pooled.append(best)
+            want = O.select_row(np.array(pooled), i, int(bud[i]), 1, 1)
+            for h in range(hk * G, (hk + 1) * G):
+                assert rows[h * nb + i] == want
+
+
+def test_group_lists_reduce_to_per_head_lists():
+    rng = np.random.default_rng(32)
+    hq, nb = 4, 7
+    cu = [0, nb * 16]
+    base = dict(block_size=16, keep_ratio=0.5, mu=0.7, sink_blocks=1, window_blocks=2)
+    sc = np.full((hq, nb, nb), -np.inf)
+    for i in range(nb):
+        sc[:, i, :i + 1] = rng.standard_normal((hq, i + 1))
+    per_head = _rows(*O.select(sc, cu, O.Params(**base))[1:])
+    # one query head per KV head: the group is the head
+    assert _rows(*O.select(sc, cu, O.Params(**base, list_mode=O.LIST_PER_GROUP), hkv=hq)[1:]) == per_head
+    # identical heads in a group: nothing to pool
+    same = np.repeat(sc[::2], 2, axis=0)
+    assert (_rows(*O.select(same, cu, O.Params(**base, list_mode=O.LIST_PER_GROUP), hkv=2)[1:])
+            == _rows(*O.select(same, cu, O.Params(**base))[1:]))
+    # a dominant head decides its group's list
+    dom = sc.copy()
+    dom[0] += 100.0
+    dom[2] += 100.0
+    grp = _rows(*O.select(dom, cu, O.Params(**base, list_mode=O.LIST_PER_GROUP), hkv=2)[1:])
+    ph = _rows(*O.select(dom, cu, O.Params(**base))[1:])
+    for i in range(nb):
+        assert grp[0 * nb + i] == grp[1 * nb + i] == ph[0 * nb + i]
+        assert grp[2 * nb + i] == grp[3 * nb + i] == ph[2 * nb + i]
+
+
 def test_oam_log_form_ranks_like_product_form():
     """HPC-BSA article §2.2: the log turns the product exp(routing) * magnitude
     into a sum without changing the ranking.  Top-k by the additive score must
