@@ -91,8 +91,8 @@ __global__ void __launch_bounds__(kBudgetThreads) budget_kernel(const SeqBatch b
       static_cast<int32_t>(static_cast<int64_t>(hq) * nnz_per_head);
 }
 
-__global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batch, int h0, int nh, int nbtot,
-                                                             int nb_max, int sink, int window,
+__global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batch, int h0, int nh, int group,
+                                                             int nbtot, int nb_max, int sink, int window,
                                                              const float* __restrict__ scores,
                                                              const int32_t* __restrict__ budgets,
                                                              const int32_t* __restrict__ row_ptr,
@@ -106,10 +106,11 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batc
   const int s = find_seq(batch, blockIdx.x);
   const int local = blockIdx.x - batch.item0[s];
   const int nb = batch.nb[s];
-  // rows of a sequence: query blocks descending (longest rows first), heads
-  // h0 .. h0 + nh - 1 inner
-  const int h = h0 + local % nh;
-  const int i = nb - 1 - local / nh;
+  // lists of a sequence: query blocks descending (longest rows first), then
+  // the lists of heads h0 .. h0 + nh - 1 (one per `group` heads)
+  const int nlists = nh / group;
+  const int h = h0 + (local % nlists) * group;  // first head of the list
+  const int i = nb - 1 - local / nlists;
   const int g = batch.g0[s] + i;
   const size_t r = static_cast<size_t>(h) * nbtot + g;
   const int c = i + 1;
@@ -118,14 +119,20 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batc
   const int ncand = c - nforced;
   const int m = min(max(b - nforced, 0), ncand);  // candidates to pick
   const float* row = scores + r * static_cast<size_t>(nb_max);
-  int32_t* out = col_idx + row_ptr[r];
+  const size_t head_stride = static_cast<size_t>(nbtot) * nb_max;  // next head's row of the same block
 
   // Threshold: the m-th largest candidate key (radix select, 8 bits per pass).
   uint32_t thr = 0u;
   int take_eq = 0;  // how many candidates equal to thr to take, lowest index first
   const bool all = (m == ncand);
   if (m > 0 && !all) {
-    for (int j = threadIdx.x; j < c; j += kSelThreads) s_key[j] = order_key(row[j]);
+    // the key of a block is that of the group's best score (order_key is
+    // monotone and maps NaN below every number)
+    for (int j = threadIdx.x; j < c; j += kSelThreads) {
+      uint32_t k = order_key(row[j]);
+      for (int e = 1; e < group; ++e) k = max(k, order_key(row[e * head_stride + j]));
+      s_key[j] = k;
+    }
     if (threadIdx.x == 0) {
       s_prefix = 0u;
       s_need = m;
@@ -198,7 +205,10 @@ __global__ void __launch_bounds__(kSelThreads) select_kernel(const SeqBatch batc
         sel = k > thr || (k == thr && e < take_eq);
         if (k == thr) ++e;
       }
-      if (sel) out[p++] = j;
+      if (sel) {
+        for (int e = 0; e < group; ++e) col_idx[row_ptr[r + static_cast<size_t>(e) * nbtot] + p] = j;
+        ++p;
+      }
     }
   }
 }
@@ -212,19 +222,20 @@ cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_
   return cudaGetLastError();
 }
 
-cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int nbtot, int nb_max, int sink, int window,
-                          const float* scores, const int32_t* budgets, const int32_t* row_ptr, int32_t* col_idx,
-                          cudaStream_t stream) {
+cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int group, int nbtot, int nb_max, int sink,
+                          int window, const float* scores, const int32_t* budgets, const int32_t* row_ptr,
+                          int32_t* col_idx, cudaStream_t stream) {
   const int items = batch.item0[batch.n];
-  if (items == 0 || nh <= 0 || h0 < 0 || h0 + nh > hq) return items == 0 || nh <= 0 ? cudaSuccess : cudaErrorInvalidValue;
+  if (items == 0 || nh <= 0) return cudaSuccess;
+  if (h0 < 0 || h0 + nh > hq || group < 1 || nh % group != 0) return cudaErrorInvalidValue;
   const size_t smem = sizeof(uint32_t) * static_cast<size_t>(nb_max);
   if (smem > 48 * 1024) {
     cudaError_t e = cudaFuncSetAttribute(select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
     if (e != cudaSuccess) return e;
   }
-  select_kernel<<<items, kSelThreads, smem, stream>>>(batch, h0, nh, nbtot, nb_max, sink, window, scores, budgets,
-                                                      row_ptr, col_idx);
+  select_kernel<<<items, kSelThreads, smem, stream>>>(batch, h0, nh, group, nbtot, nb_max, sink, window, scores,
+                                                      budgets, row_ptr, col_idx);
   return cudaGetLastError();
 }
 

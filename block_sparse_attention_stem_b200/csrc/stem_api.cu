@@ -60,6 +60,7 @@ stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
   if (!(p->softmax_scale >= 0.0) || !std::isfinite(p->softmax_scale)) return STEM_ERR_INVALID_ARG;
   if (p->budget_mode != STEM_BUDGET_RELATIVE && p->budget_mode != STEM_BUDGET_ABSOLUTE) return STEM_ERR_INVALID_ARG;
   if (p->bonus_mode != STEM_BONUS_LOG && p->bonus_mode != STEM_BONUS_STANDARDIZED) return STEM_ERR_INVALID_ARG;
+  if (p->list_mode != STEM_LIST_PER_HEAD && p->list_mode != STEM_LIST_PER_GROUP) return STEM_ERR_INVALID_ARG;
   return STEM_OK;
 }
 
@@ -285,8 +286,11 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
                                                  row_ptr, stream));
     if (st != STEM_OK) return st;
   }
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * G * si.nb; })) {
-    stem_status_t st = cuda_status(launch_select(b, hq, hk0 * G, nhk * G, nbtot, nb_max, p->sink_blocks,
+  // one CTA per list: per (query head, query block), or per (KV head, query
+  // block) when the query heads of a group share their lists
+  const int per_list = p->list_mode == STEM_LIST_PER_GROUP ? G : 1;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * (G / per_list) * si.nb; })) {
+    stem_status_t st = cuda_status(launch_select(b, hq, hk0 * G, nhk * G, per_list, nbtot, nb_max, p->sink_blocks,
                                                  p->window_blocks, scores,
                                                  budgets, row_ptr, col_idx, stream));
     if (st != STEM_OK) return st;

@@ -66,8 +66,11 @@ cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const Sco
                          cudaStream_t stream);
 cudaError_t launch_budget(const SeqBatch& batch, int hq, int nbtot, int64_t nnz_per_head, double rho, double mu,
                           int sink, int window, int mode, int32_t* budgets, int32_t* row_ptr, cudaStream_t stream);
-// rows of query heads h0 .. h0 + nh - 1 only (batch items: nh * nb per sequence)
-cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int nbtot, int nb_max, int sink, int window,
+// rows of query heads h0 .. h0 + nh - 1 only; `group` consecutive heads share
+// one list selected on the max of their scores (batch items: nh / group * nb
+// per sequence)
+cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int group, int nbtot, int nb_max, int sink,
+                          int window,
                           const float* scores, const int32_t* budgets, const int32_t* row_ptr, int32_t* col_idx,
                           cudaStream_t stream);
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,

@@ -54,12 +54,14 @@ class Workload:
     softmax_scale: float = 0.0
     budget_mode: int = 0
     bonus_mode: int = 0
+    list_mode: int = 0
 
     def params(self) -> dict:
         return dict(block_size=self.block_size, stride=self.stride, chunk_size=self.chunk_size,
                     norm=self.norm, beta=self.beta, keep_ratio=self.keep_ratio, mu=self.mu,
                     sink_blocks=self.sink_blocks, window_blocks=self.window_blocks,
-                    softmax_scale=self.softmax_scale, budget_mode=self.budget_mode, bonus_mode=self.bonus_mode)
+                    softmax_scale=self.softmax_scale, budget_mode=self.budget_mode, bonus_mode=self.bonus_mode,
+                    list_mode=self.list_mode)
 
     @property
     def total_tokens(self) -> int:

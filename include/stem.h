@@ -84,6 +84,14 @@ typedef enum {
                                   the statistics' scope is this library's reading] */
 } stem_bonus_mode_t;
 
+/* Granularity of the block lists under GQA. */
+typedef enum {
+  STEM_LIST_PER_HEAD = 0,  /* every query head selects its own blocks */
+  STEM_LIST_PER_GROUP = 1  /* one list per (KV head, query block), selected on the
+                              elementwise max of its query heads' scores (NaN as
+                              -inf) and written to every query head of the group */
+} stem_list_mode_t;
+
 /* Method parameters (AngelSlim documentation §6 defaults in brackets). */
 typedef struct {
   int32_t block_size;     /* attention block [128]; only 128 is supported */
@@ -98,6 +106,7 @@ typedef struct {
   double  softmax_scale;  /* attention logit scale; 0 selects 1/sqrt(head_dim) */
   int32_t budget_mode;    /* stem_budget_mode_t */
   int32_t bonus_mode;     /* stem_bonus_mode_t [STEM_BONUS_LOG] */
+  int32_t list_mode;      /* stem_list_mode_t [STEM_LIST_PER_HEAD] */
 } stem_params_t;
 
 /* Query/key/value description shared by all calls. */
@@ -169,6 +178,8 @@ STEM_API stem_status_t stem_score(const stem_qkv_t* qkv, const stem_params_t* pa
  *   b = min(c, max(k, |F|))
  *   row = F u the b-|F| best other causal blocks by (score desc, index asc),
  *         NaN ranked as -inf, written in ascending order.
+ * STEM_LIST_PER_GROUP: the rows of the G query heads of a KV head share one list,
+ *         selected on the elementwise max of their score rows.
  * Outputs: budgets int32 [Hq*NBtot], row_ptr int32 [Hq*NBtot + 1] (row_ptr[0] = 0),
  * col_idx int32 [nnz] (key-block indices local to the sequence). */
 STEM_API stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params,

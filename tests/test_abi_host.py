@@ -114,6 +114,8 @@ def test_validation_rejects_bad_parameters():
     assert _status(lambda: b.stem_plan(qkv, P(budget_mode=2))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(bonus_mode=2))) == 1
     b.stem_plan(qkv, P(bonus_mode=1))  # the standardized bonus is valid
+    assert _status(lambda: b.stem_plan(qkv, P(list_mode=2))) == 1
+    b.stem_plan(qkv, P(list_mode=1))  # GQA-shared lists are valid
     assert _status(lambda: b.stem_plan(qkv, P(stride=3))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(stride=16))) == 2
     assert _status(lambda: b.stem_plan(qkv, P(block_size=64))) == 2

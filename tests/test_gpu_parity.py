@@ -45,6 +45,9 @@ CASES = {
     # standardized value bonus (per-sequence, per-KV-head z-score of ln ||v||^2)
     "std_bonus_varlen": W([1000, 128, 2088], 8, 2, seed=19, bonus_mode=1),
     "std_bonus_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=20, bonus_mode=1),
+    # one block list per KV head (max over its query heads), shared by the group
+    "group_lists": W([1000, 128, 2088], 8, 2, seed=21, list_mode=1),
+    "group_lists_odd_group": W([1500, 700], 6, 2, seed=22, list_mode=1, keep_ratio=0.25),
 }
 
 
@@ -92,7 +95,7 @@ def test_select_is_bit_exact_on_identical_fp32_scores(name):
     s32 = c.ref_scores.astype(np.float32)
     gb, grp, gci, ws = b.stem_select(c.qkv, c.params, torch.from_numpy(s32).cuda())
     assert b.stem_read_device_status(ws) == 0
-    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p)
+    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p, hkv=c.w.num_kv_heads)
     assert np.array_equal(gb.cpu().numpy(), ob)
     assert np.array_equal(grp.cpu().numpy(), orp)
     assert np.array_equal(gci.cpu().numpy(), oci)
@@ -104,7 +107,7 @@ def test_select_ties_go_to_lowest_index():
     s32 = np.round(c.ref_scores * 2).astype(np.float32) / 2  # many exact ties
     s32[rng.random(s32.shape) < 0.05] = np.nan               # NaN ranks as -inf
     gb, grp, gci, _ = b.stem_select(c.qkv, c.params, torch.from_numpy(s32).cuda())
-    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p)
+    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p, hkv=c.w.num_kv_heads)
     assert np.array_equal(grp.cpu().numpy(), orp)
     assert np.array_equal(gci.cpu().numpy(), oci)
 
@@ -115,8 +118,9 @@ def test_prefill_end_to_end(name):
     out, lse, rp, ci, ws = b.stem_prefill(c.qkv, c.params)
     assert b.stem_read_device_status(ws) == 0
     rp, ci = rp.cpu().numpy(), ci.cpu().numpy()
-    ob, orp, oci = O.select(c.ref_scores, c.cu, c.p)
-    compare_lists(rp, ci, orp, oci, c.ref_scores, c.cu, c.w.num_q_heads, c.p.sink_blocks, c.p.window_blocks)
+    ob, orp, oci = O.select(c.ref_scores, c.cu, c.p, hkv=c.w.num_kv_heads)
+    ranked = O.group_pooled_scores(c.ref_scores, c.w.num_kv_heads) if c.p.list_mode else c.ref_scores
+    compare_lists(rp, ci, orp, oci, ranked, c.cu, c.w.num_q_heads, c.p.sink_blocks, c.p.window_blocks)
     # attention with the GPU's own lists
     ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp, ci, c.p)
     check_attention(out, lse, ro, rl, c.w.dtype)
