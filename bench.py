@@ -54,9 +54,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
-    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality"], default="default",
+    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality", "variants"], default="default",
                     help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack; "
-                         "quality: reconstruction error against dense attention (32K)")
+                         "quality: reconstruction error against dense attention (32K); "
+                         "variants: the 128K step with the standardized bonus and KV-group-shared lists")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
     return ap.parse_args(argv)
 
@@ -486,7 +487,7 @@ def run_reference(args):
 
 
 # ---------------------------------------------------------------- extra modes (one GPU)
-def _time_prefill(b, qkv, params, pl, dev, steps, warmup):
+def _time_prefill(b, qkv, params, pl, dev, steps, warmup, stages=None):
     """Mean CUDA-event time (ms) of the three stages and of the attention
     stage alone over `steps` runs after `warmup`."""
     import torch
@@ -515,6 +516,10 @@ def _time_prefill(b, qkv, params, pl, dev, steps, warmup):
         raise RuntimeError(b.stem_status_string(status))
     tot = sum(e[0].elapsed_time(e[3]) for e in ev[warmup:]) / steps
     bsa = sum(e[2].elapsed_time(e[3]) for e in ev[warmup:]) / steps
+    if stages is not None:
+        stages["score"] = sum(e[0].elapsed_time(e[1]) for e in ev[warmup:]) / steps
+        stages["select"] = sum(e[1].elapsed_time(e[2]) for e in ev[warmup:]) / steps
+        stages["bsa"] = bsa
     return tot, bsa
 
 
@@ -599,7 +604,9 @@ def run_quality(args):
     for label, kw in (("stem: OAM beta 0.2, TPD mu 0.7", dict(beta=0.2, mu=0.7)),
                       ("routing score only: beta 0, mu 0.7", dict(beta=0.0, mu=0.7)),
                       ("OAM beta 0.2, uniform budget mu 1 (same kept blocks)", dict(beta=0.2, mu=1.0, keep_ratio=rho_eq)),
-                      ("routing score only, uniform budget", dict(beta=0.0, mu=1.0, keep_ratio=rho_eq))):
+                      ("routing score only, uniform budget", dict(beta=0.0, mu=1.0, keep_ratio=rho_eq)),
+                      ("standardized bonus beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, bonus_mode=1)),
+                      ("KV-group-shared lists, beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, list_mode=1))):
         params = b.make_params(**dict(w0.params(), **kw))
         out, lse, _, _, ws = b.stem_prefill(qkv, params, return_lists=False)
         torch.cuda.synchronize()
@@ -611,6 +618,36 @@ def run_quality(args):
                            rel_error_vs_dense=round(err, 5), softmax_mass_kept=round(mass, 5), **kw))
     res = {"metric": "attention reconstruction vs dense (32K, synthetic)", "unit": "relative Frobenius error",
            "higher_is_better": False, "points": points, "config": describe(w0), "dtype": "bf16",
+           "data": "synthetic (seeded, device RNG)"}
+    print(json.dumps(res), flush=True)
+
+
+def run_variants(args):
+    """The step on the 128K workload with the selection variants beside the
+    default: the standardized value bonus (bonus_mode 1) and KV-group-shared
+    block lists (list_mode 1); ms per stage and attention TFLOP/s."""
+    import torch
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+    dev = torch.device("cuda", 0)
+    w0 = I.workload("long128k")
+    inp = I.make_inputs(w0, device="cuda")
+    qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w0.cu_seqlens(), cu_seqlens_dev=inp["cu_seqlens"])
+    rows = []
+    sampler = ClockSampler(gpu_device_id(torch))
+    sampler.start()
+    for label, kw in (("default (log bonus, per-head lists)", {}),
+                      ("standardized bonus (bonus_mode 1)", dict(bonus_mode=1)),
+                      ("KV-group-shared lists (list_mode 1)", dict(list_mode=1))):
+        params = b.make_params(**dict(w0.params(), **kw))
+        pl = b.stem_plan(qkv, params)
+        st = {}
+        tot, bsa = _time_prefill(b, qkv, params, pl, dev, args.steps, args.warmup, stages=st)
+        rows.append(dict(variant=label, ms=round(tot, 3), stages_ms={k: round(v, 3) for k, v in st.items()},
+                         attn_tflops=round(pl.attn_flops / (bsa * 1e-3) / 1e12, 1), **kw))
+    clocks = sampler.stop()
+    res = {"metric": "128K step per selection variant", "unit": "ms", "higher_is_better": False, "points": rows,
+           "steps": args.steps, "warmup": args.warmup, "config": describe(w0), "clocks": clocks, "dtype": "bf16",
            "data": "synthetic (seeded, device RNG)"}
     print(json.dumps(res), flush=True)
 
@@ -656,6 +693,8 @@ def main(argv=None):
         run_sweep(args)
     elif args.mode == "quality":
         run_quality(args)
+    elif args.mode == "variants":
+        run_variants(args)
     elif args.mode == "fp8stack":
         run_fp8stack(args)
     else:
