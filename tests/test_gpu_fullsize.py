@@ -150,3 +150,14 @@ def test_fullsize_fp8_varlen_layers(layer):
 def test_fullsize_sweep64k_extremes(rho):
     w = I.workload("sweep64k", keep_ratio=rho)
     _check_workload(w, _samples(w, (7,), lambda nb: (2, nb - 1)))
+
+
+def test_rows_longer_than_the_staged_list():
+    """Rows with more than 2048 listed blocks (the attention kernel stages at
+    most 2048 list entries in shared memory and walks longer lists in global
+    memory): one 270K-token sequence at keep ratio 0.99 with a uniform budget."""
+    nb = 2112
+    w = I.Workload(name="long_rows", seqlens=[nb * 128], num_q_heads=2, num_kv_heads=1, seed=41, keep_ratio=0.99,
+                   mu=1.0, beta=0.2, sink_blocks=1, window_blocks=2)
+    assert O.budgets(w.cu_seqlens(), O.Params(**w.params()))[-1] > 2048
+    _check_workload(w, [(0, 0, nb - 1), (0, 1, nb - 40)])
