@@ -533,6 +533,21 @@ def full_csr(cu_seqlens, hq: int, block: int = 128):
     return row_ptr, col_idx
 
 
+def gather_paged(pages: np.ndarray, page_table: np.ndarray, cu_seqlens, page_size: int) -> np.ndarray:
+    """Paged KV (AngelSlim doc's paged fp8 KV path for the block-sparse
+    attention): the keys (or values) of sequence s, token t, live at
+    pages[page_table[s][t // page_size], t % page_size].  pages [P, page_size,
+    H, d]; page_table [num_seqs, max_pages] int.  Returns the packed [T, H, d]
+    tensor that the contiguous path reads, which is all the paged path means:
+    attention over paged K/V equals attention over this gather."""
+    T = cu_seqlens[-1]
+    out = np.empty((T,) + pages.shape[2:], dtype=pages.dtype)
+    for s in range(len(cu_seqlens) - 1):
+        for t in range(cu_seqlens[s + 1] - cu_seqlens[s]):
+            out[cu_seqlens[s] + t] = pages[page_table[s][t // page_size], t % page_size]
+    return out
+
+
 def prefill(q, k, v, cu_seqlens, p: Params):
     """score -> select -> block-sparse attention, all in fp64."""
     S = block_scores(q, k, v, cu_seqlens, p)

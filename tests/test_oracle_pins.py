@@ -366,6 +366,28 @@ def test_group_lists_reduce_to_per_head_lists():
         assert grp[2 * nb + i] == grp[3 * nb + i] == ph[2 * nb + i]
 
 
+def test_paged_gather_is_the_page_table_lookup():
+    rng = np.random.default_rng(41)
+    cu, ps = [0, 150, 150 + 64, 150 + 64 + 1], 64
+    kc = rng.standard_normal((cu[-1], 2, 4))
+    # contiguous pages in order reproduce the packed tensor ...
+    npg = [(cu[i + 1] - cu[i] + ps - 1) // ps for i in range(3)]
+    pages = np.zeros((sum(npg), ps, 2, 4))
+    table = np.zeros((3, max(npg)), dtype=np.int64)
+    nxt = 0
+    for sq in range(3):
+        for pg in range(npg[sq]):
+            n = min(ps, cu[sq + 1] - cu[sq] - pg * ps)
+            pages[nxt, :n] = kc[cu[sq] + pg * ps: cu[sq] + pg * ps + n]
+            table[sq, pg] = nxt
+            nxt += 1
+    assert np.array_equal(O.gather_paged(pages, table, cu, ps), kc)
+    # ... and so does any permutation of the pool with the table permuted alike
+    perm = rng.permutation(len(pages))
+    inv = np.argsort(perm)
+    assert np.array_equal(O.gather_paged(pages[perm], inv[table], cu, ps), kc)
+
+
 def test_oam_log_form_ranks_like_product_form():
     """HPC-BSA article §2.2: the log turns the product exp(routing) * magnitude
     into a sum without changing the ranking.  Top-k by the additive score must
