@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "STEM_OK", 1: "STEM_ERR_INVALID_ARG", 2: "STEM_ERR_UNSUPPORTE
                 3: "STEM_ERR_WORKSPACE_TOO_SMALL", 4: "STEM_ERR_MISALIGNED", 5: "STEM_ERR_CUDA",
                 6: "STEM_ERR_TIMEOUT", 7: "STEM_ERR_BAD_BLOCKLIST"}
 STEM_BF16, STEM_FP8_E4M3 = 0, 1
-EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill", "stem_prefill_host",
+EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_bsa_fwd_paged", "stem_prefill",
+            "stem_prefill_host",
             "stem_prefill_noalloc",
             "stem_selftest_wait_timeout", "stem_read_device_status", "stem_status_string", "stem_version")
 
@@ -44,6 +45,11 @@ class StemQKV(ctypes.Structure):
                 ("num_q_heads", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("q", ctypes.c_void_p), ("k", ctypes.c_void_p), ("v", ctypes.c_void_p),
                 ("q_scale", ctypes.c_void_p), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p)]
+
+
+class StemPagedKV(ctypes.Structure):
+    _fields_ = [("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("page_table", ctypes.c_void_p), ("k_pages", ctypes.c_void_p), ("v_pages", ctypes.c_void_p)]
 
 
 class StemPlan(ctypes.Structure):
@@ -70,6 +76,7 @@ def _load() -> ctypes.CDLL:
     lib.stem_score.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, sz, vp]
     lib.stem_select.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_bsa_fwd.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
+    lib.stem_bsa_fwd_paged.argtypes = [P(StemQKV), P(StemPagedKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill_noalloc.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp]
     lib.stem_prefill_host.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -194,6 +201,44 @@ def stem_select(qkv: QKV, params: StemParams, scores, budgets=None, row_ptr=None
     _check(LIB.stem_select(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(scores), _ptr(budgets),
                            _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(), _stream(stream)), "stem_select")
     return budgets, row_ptr, col_idx[:pl.nnz], ws
+
+
+@dataclass
+class PagedKV:
+    """A paged K/V pool and the descriptor that points at it; keeps the
+    tensors alive while the descriptor is used."""
+    k_pages: torch.Tensor
+    v_pages: torch.Tensor
+    page_table: torch.Tensor
+    desc: StemPagedKV
+
+
+def paged_kv(k_pages, v_pages, page_table, page_size: int) -> PagedKV:
+    """k_pages/v_pages [P, page_size, Hkv, d] device tensors, page_table int32
+    [num_seqs, max_pages] on the device."""
+    if page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_contiguous():
+        raise ValueError("page_table must be a contiguous int32 [num_seqs, max_pages] tensor")
+    if k_pages.shape != v_pages.shape or k_pages.shape[1] != page_size:
+        raise ValueError("k_pages and v_pages must both be [P, page_size, Hkv, d]")
+    desc = StemPagedKV(page_size, k_pages.shape[0], page_table.shape[1], _ptr(page_table), _ptr(k_pages),
+                       _ptr(v_pages))
+    return PagedKV(k_pages, v_pages, page_table, desc)
+
+
+def stem_bsa_fwd_paged(qkv: QKV, kv: PagedKV, params: StemParams, row_ptr, col_idx, out=None, lse=None,
+                       ws=None, stream=None):
+    pl = stem_plan(qkv, params)
+    dev = qkv.q.device
+    T, hq = qkv.total_tokens, qkv.q.shape[1]
+    if out is None:
+        out = torch.empty(T, hq, 128, dtype=torch.bfloat16, device=dev)
+    if lse is None:
+        lse = torch.empty(hq, T, dtype=torch.float32, device=dev)
+    ws = _ws(pl.ws_bytes, dev, ws)
+    _check(LIB.stem_bsa_fwd_paged(ctypes.byref(qkv.desc), ctypes.byref(kv.desc), ctypes.byref(params), _ptr(row_ptr),
+                                  _ptr(col_idx), _ptr(out), _ptr(lse), _ptr(ws), ws.numel(), _stream(stream)),
+           "stem_bsa_fwd_paged")
+    return out, lse, ws
 
 
 def stem_bsa_fwd(qkv: QKV, params: StemParams, row_ptr, col_idx, out=None, lse=None, ws=None, stream=None):

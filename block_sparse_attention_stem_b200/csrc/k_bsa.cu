@@ -249,7 +249,9 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
     // ------------------------------------------------------------ producers
     const bool is_v = warp == kVProducerWarp;
     if (lane == 0 && N > 0) {
-      const CUtensorMap* m = is_v ? &maps.v[seq] : &maps.k[seq];
+      const bool paged = args.page_table != nullptr;
+      const CUtensorMap* m = paged ? (is_v ? &maps.v_pool : &maps.k_pool) : (is_v ? &maps.v[seq] : &maps.k[seq]);
+      const int32_t* pages = paged ? args.page_table + static_cast<size_t>(batch.seq_id[seq]) * args.max_pages : nullptr;
       tma_prefetch_desc(m);
       if (!is_v) {
         mbar_arrive_expect_tx(&sm.q_full, Cfg::kQBytes);
@@ -267,9 +269,13 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
         if ((h & 1) == 0) j = cur.next(sm.list, list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
         uint8_t* dst = is_v ? sm.v[h & 1] : sm.k[h & 1];
         uint64_t* bar = is_v ? &sm.v_full[h & 1] : &sm.k_full[h & 1];
+        // token row of the half: in the sequence, or through the page table (a
+        // 64-key half never straddles a page; a page number outside the pool
+        // reads zeros)
+        int row = j * kBlock + (h & 1) * kHalf;
+        if (paged) row = __ldg(pages + row / args.page_size) * args.page_size + row % args.page_size;
         mbar_arrive_expect_tx(bar, Cfg::kHalfBytes);
-        for (int hh = 0; hh < kSlabs; ++hh)
-          tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, j * kBlock + (h & 1) * kHalf);
+        for (int hh = 0; hh < kSlabs; ++hh) tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, row);
         ++issued;
       }
       // every copy of this producer has landed before the CTA can exit (a

@@ -145,6 +145,7 @@ std::vector<SeqBatch> make_batches(const Plan& pl, F items) {
       b.nb[q] = si.nb;
       b.g0[q] = si.g0;
       b.csr0[q] = si.csr0;
+      b.seq_id[q] = si.idx;
       b.item0[q + 1] = b.item0[q] + items(si);
     }
     for (int q = b.n; q < kMaxSeqPerLaunch; ++q) b.item0[q + 1] = b.item0[q];
@@ -299,8 +300,8 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
 }
 
 stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
-                      const int32_t* row_ptr,
-                      const int32_t* col_idx, void* out, float* lse, int* status, cudaStream_t stream) {
+                      const int32_t* row_ptr, const int32_t* col_idx, void* out, float* lse, int* status,
+                      cudaStream_t stream, const stem_paged_kv_t* paged = nullptr) {
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
   BsaArgs a{};
@@ -319,17 +320,27 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.lse = lse;
   a.status = status;
   a.hk0 = hk0;
+  BsaMaps maps;
+  std::memset(&maps, 0, sizeof(maps));
+  if (paged) {
+    // the page pool as one token sequence of pages * page_size rows
+    const int pool = paged->num_pages * paged->page_size;
+    if (!encode_seq_map(&maps.k_pool, paged->k_pages, fp8, hkv, 0, pool, kBlock / 2, 1) ||
+        !encode_seq_map(&maps.v_pool, paged->v_pages, fp8, hkv, 0, pool, kBlock / 2, 1))
+      return STEM_ERR_CUDA;
+    a.page_table = paged->page_table;
+    a.page_size = paged->page_size;
+    a.max_pages = paged->max_pages_per_seq;
+  }
   // one CTA per CSR row (query head, query block)
   const int G = hq / hkv;
   for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * G * si.nb; })) {
-    BsaMaps maps;
-    std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
       // Q in 128-token boxes; K and V in 64-token boxes (the attention
       // kernel moves half a key block per copy)
-      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1) ||
-          !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1) ||
-          !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1))
+      if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1)) return STEM_ERR_CUDA;
+      if (!paged && (!encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1) ||
+                     !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1)))
         return STEM_ERR_CUDA;
     }
     stem_status_t st = cuda_status(launch_bsa(maps, b, a, fp8, stream));
@@ -394,6 +405,36 @@ stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params, c
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
   return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s);
+}
+
+stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_paged_kv_t* kv, const stem_params_t* params,
+                                 const int32_t* row_ptr, const int32_t* col_idx, void* out, float* lse, void* ws,
+                                 size_t ws_bytes, stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if (!kv) return STEM_ERR_INVALID_ARG;
+  if (qkv->total_tokens > 0) {
+    if (!qkv->q || !qkv->cu_seqlens || !kv->k_pages || !kv->v_pages || !kv->page_table) return STEM_ERR_INVALID_ARG;
+    if (!aligned16(qkv->q) || !aligned16(kv->k_pages) || !aligned16(kv->v_pages)) return STEM_ERR_MISALIGNED;
+  }
+  if (qkv->dtype == STEM_FP8_E4M3 && (!qkv->q_scale || !qkv->k_scale || !qkv->v_scale)) return STEM_ERR_INVALID_ARG;
+  // a 64-key half must sit inside one page, and every token needs a page
+  if (kv->page_size < 64 || kv->page_size % 64 != 0 || kv->num_pages < 1 || kv->max_pages_per_seq < 1)
+    return STEM_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(kv->num_pages) * kv->page_size > INT32_MAX) return STEM_ERR_INVALID_ARG;
+  for (int q = 0; q < qkv->num_seqs; ++q) {
+    const int64_t L = qkv->cu_seqlens_host[q + 1] - qkv->cu_seqlens_host[q];
+    // the last key block may run past L to its 128-token end
+    const int64_t need = (L + kBlock - 1) / kBlock * kBlock;
+    if (need > static_cast<int64_t>(kv->max_pages_per_seq) * kv->page_size) return STEM_ERR_INVALID_ARG;
+  }
+  if (!row_ptr || !col_idx || !out || !lse || !ws) return STEM_ERR_INVALID_ARG;
+  if (!aligned16(out)) return STEM_ERR_MISALIGNED;
+  if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s, kv);
 }
 
 stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, void* out, float* lse,

@@ -32,6 +32,7 @@ struct SeqBatch {
   int32_t g0[kMaxSeqPerLaunch];       // global index of the sequence's block 0
   int32_t item0[kMaxSeqPerLaunch + 1];
   int64_t csr0[kMaxSeqPerLaunch];     // CSR offset of the sequence's first row inside one head
+  int32_t seq_id[kMaxSeqPerLaunch];   // the sequence's number in the call (cu_seqlens order)
 };
 
 STEM_HD int find_seq(const SeqBatch& b, int item) {

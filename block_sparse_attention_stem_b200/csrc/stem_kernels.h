@@ -24,8 +24,10 @@ struct ScoreMaps {
 
 struct BsaMaps {
   CUtensorMap q[kMaxSeqPerLaunch];  // box 128 tokens
-  CUtensorMap k[kMaxSeqPerLaunch];
+  CUtensorMap k[kMaxSeqPerLaunch];  // box 64 tokens (unused when K/V are paged)
   CUtensorMap v[kMaxSeqPerLaunch];
+  CUtensorMap k_pool;               // paged K/V: the whole page pool as [pages * page_size] tokens
+  CUtensorMap v_pool;
 };
 
 struct ScoreArgs {
@@ -42,6 +44,9 @@ struct ScoreArgs {
 struct BsaArgs {
   int hq, hkv, nbtot, total_tokens;
   int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
+  const int32_t* page_table;  // paged K/V: [num_seqs][max_pages] physical page per logical page, else null
+  int page_size;            // tokens per page, a multiple of 64
+  int max_pages;            // row length of page_table
   float scale_log2;         // softmax scale * log2(e)
   const float* q_scale;     // fp8 only
   const float* k_scale;

@@ -128,6 +128,20 @@ typedef struct {
   const float* v_scale;           /* fp8 only: device [Hkv] */
 } stem_qkv_t;
 
+/* K and V in a page pool instead of packed storage (the paged fp8 KV path of
+ * AngelSlim doc §5; bf16 pages work the same way).  Token t of sequence s is
+ * row t % page_size of page page_table[s * max_pages_per_seq + t / page_size];
+ * each row is [Hkv, d] like a packed token row. */
+typedef struct {
+  int32_t page_size;          /* tokens per page; a multiple of 64 */
+  int32_t num_pages;          /* pages in the pool (num_pages * page_size < 2^31) */
+  int32_t max_pages_per_seq;  /* row length of page_table; pages must cover every
+                                 sequence rounded up to a multiple of 128 tokens */
+  const int32_t* page_table;  /* device int32 [num_seqs][max_pages_per_seq] */
+  const void* k_pages;        /* device [num_pages, page_size, Hkv, d] bf16 or e4m3 bytes */
+  const void* v_pages;        /* device, same shape */
+} stem_paged_kv_t;
+
 /* Sizes derived on the host from (cu_seqlens_host, params); data-independent. */
 typedef struct {
   int64_t nb_total;          /* NBtot */
@@ -200,6 +214,20 @@ STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* 
                            const int32_t* row_ptr, const int32_t* col_idx,
                            void* out, float* lse,
                            void* ws, size_t ws_bytes, stem_stream_t stream);
+
+/* stem_bsa_fwd with K and V read through a page table (qkv->k and qkv->v are
+ * not used and may be NULL; q, cu_seqlens and the fp8 scales as for
+ * stem_bsa_fwd).  Results equal stem_bsa_fwd's on the packed K/V the pages
+ * hold, bit for bit.  Page rows past a sequence's last token (up to its next
+ * multiple of 128) are read: they must hold finite values, zeros for example.
+ * A page number outside [0, num_pages) reads zeros.  STEM_ERR_INVALID_ARG for
+ * a page size that is not a positive multiple of 64 or a table too short for
+ * some sequence. */
+STEM_API stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_paged_kv_t* kv,
+                                 const stem_params_t* params,
+                                 const int32_t* row_ptr, const int32_t* col_idx,
+                                 void* out, float* lse,
+                                 void* ws, size_t ws_bytes, stem_stream_t stream);
 
 /* score -> select -> attention on one stream with no host round trip.
  * row_ptr_out / col_idx_out may be NULL (the workspace then holds the lists);

@@ -150,6 +150,25 @@ def test_validation_rejects_bad_shapes_and_pointers():
     assert code == 1
 
 
+def test_paged_kv_validation():
+    qkv = fake_qkv([1000, 300], 4, 2)
+    P = b.make_params()
+    fake = 1 << 20  # never dereferenced: validation fails first
+
+    def kv(page_size, num_pages, max_pages):
+        return b.StemPagedKV(page_size, num_pages, max_pages, fake, fake, fake)
+
+    def call(d):  # straight through the C ABI: no device memory is touched
+        return b.LIB.stem_bsa_fwd_paged(ctypes.byref(qkv.desc), ctypes.byref(d), ctypes.byref(P), None, None, None,
+                                        None, None, 0, None)
+
+    assert call(kv(96, 64, 16)) == 1   # not a multiple of 64
+    assert call(kv(0, 64, 16)) == 1
+    assert call(kv(128, 64, 7)) == 1   # 1000 tokens need 8 pages of 128
+    assert call(kv(64, 0, 16)) == 1
+    assert call(kv(128, 64, 8)) == 1   # valid pages, but no lists: rejected too
+
+
 def test_workspace_too_small_is_reported_before_launch():
     qkv = fake_qkv([4096], 4, 2)
     P = b.make_params()
