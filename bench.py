@@ -645,6 +645,37 @@ def run_variants(args):
         tot, bsa = _time_prefill(b, qkv, params, pl, dev, args.steps, args.warmup, stages=st)
         rows.append(dict(variant=label, ms=round(tot, 3), stages_ms={k: round(v, 3) for k, v in st.items()},
                          attn_tflops=round(pl.attn_flops / (bsa * 1e-3) / 1e12, 1), **kw))
+    # the default lists with K/V in a page pool (128-token pages in a random
+    # order) against the packed layout: attention alone
+    params = b.make_params(**w0.params())
+    pl = b.stem_plan(qkv, params)
+    _, _, rp, ci, _ = b.stem_prefill(qkv, params)
+    ps = 128
+    npg = w0.total_tokens // ps
+    perm = torch.randperm(npg, generator=torch.Generator().manual_seed(5)).cuda()
+    kp = torch.empty(npg, ps, w0.num_kv_heads, 128, dtype=inp["k"].dtype, device=dev)
+    vp = torch.empty_like(kp)
+    kp[perm] = inp["k"].view(npg, ps, w0.num_kv_heads, 128)
+    vp[perm] = inp["v"].view(npg, ps, w0.num_kv_heads, 128)
+    kv = b.paged_kv(kp, vp, perm.to(torch.int32).view(1, npg).contiguous(), ps)
+    out = torch.empty(w0.total_tokens, w0.num_q_heads, 128, dtype=torch.bfloat16, device=dev)
+    lse = torch.empty(w0.num_q_heads, w0.total_tokens, dtype=torch.float32, device=dev)
+    ws = torch.empty(pl.ws_bytes, dtype=torch.uint8, device=dev)
+    for paged in (False, True):
+        for _ in range(args.warmup):
+            (b.stem_bsa_fwd_paged(qkv, kv, params, rp, ci, out, lse, ws) if paged
+             else b.stem_bsa_fwd(qkv, params, rp, ci, out, lse, ws))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            (b.stem_bsa_fwd_paged(qkv, kv, params, rp, ci, out, lse, ws) if paged
+             else b.stem_bsa_fwd(qkv, params, rp, ci, out, lse, ws))
+        e1.record()
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / args.steps
+        rows.append(dict(variant=("attention over paged K/V (128-token pages, shuffled)" if paged
+                                  else "attention over packed K/V"), ms=round(ms, 3),
+                         attn_tflops=round(pl.attn_flops / (ms * 1e-3) / 1e12, 1)))
     clocks = sampler.stop()
     res = {"metric": "128K step per selection variant", "unit": "ms", "higher_is_better": False, "points": rows,
            "steps": args.steps, "warmup": args.warmup, "config": describe(w0), "clocks": clocks, "dtype": "bf16",
