@@ -25,7 +25,8 @@ STATUS_NAMES = {0: "STEM_OK", 1: "STEM_ERR_INVALID_ARG", 2: "STEM_ERR_UNSUPPORTE
                 3: "STEM_ERR_WORKSPACE_TOO_SMALL", 4: "STEM_ERR_MISALIGNED", 5: "STEM_ERR_CUDA",
                 6: "STEM_ERR_TIMEOUT", 7: "STEM_ERR_BAD_BLOCKLIST"}
 STEM_BF16, STEM_FP8_E4M3 = 0, 1
-EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_bsa_fwd_paged", "stem_prefill",
+EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_score_select", "stem_bsa_fwd", "stem_bsa_fwd_paged",
+            "stem_prefill",
             "stem_prefill_host",
             "stem_prefill_noalloc",
             "stem_selftest_wait_timeout", "stem_read_device_status", "stem_status_string", "stem_version")
@@ -75,6 +76,7 @@ def _load() -> ctypes.CDLL:
     lib.stem_plan.argtypes = [P(StemQKV), P(StemParams), P(StemPlan)]
     lib.stem_score.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, sz, vp]
     lib.stem_select.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
+    lib.stem_score_select.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, vp, sz, vp]
     lib.stem_bsa_fwd.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_bsa_fwd_paged.argtypes = [P(StemQKV), P(StemPagedKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
@@ -201,6 +203,27 @@ def stem_select(qkv: QKV, params: StemParams, scores, budgets=None, row_ptr=None
     _check(LIB.stem_select(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(scores), _ptr(budgets),
                            _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(), _stream(stream)), "stem_select")
     return budgets, row_ptr, col_idx[:pl.nnz], ws
+
+
+def stem_score_select(qkv: QKV, params: StemParams, scores=None, vbonus=None, budgets=None, row_ptr=None,
+                      col_idx=None, ws=None, stream=None):
+    """stem_score then stem_select in one pass (the scoring CTAs select their rows)."""
+    pl = stem_plan(qkv, params)
+    dev = qkv.q.device
+    hq, hkv = qkv.q.shape[1], qkv.k.shape[1]
+    if scores is None:
+        scores = torch.empty(hq, pl.nb_total, pl.nb_max, dtype=torch.float32, device=dev)
+    if budgets is None:
+        budgets = torch.empty(pl.num_rows, dtype=torch.int32, device=dev)
+    if row_ptr is None:
+        row_ptr = torch.empty(pl.num_rows + 1, dtype=torch.int32, device=dev)
+    if col_idx is None:
+        col_idx = torch.empty(max(pl.nnz, 1), dtype=torch.int32, device=dev)
+    ws = _ws(pl.ws_bytes, dev, ws)
+    _check(LIB.stem_score_select(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(scores), _ptr(vbonus),
+                                 _ptr(budgets), _ptr(row_ptr), _ptr(col_idx), _ptr(ws), ws.numel(),
+                                 _stream(stream)), "stem_score_select")
+    return scores, budgets, row_ptr, col_idx[:pl.nnz], ws
 
 
 @dataclass

@@ -29,6 +29,7 @@
 // owner + MMA issuer.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
+#include "stem_select_row.cuh"
 
 namespace stem {
 
@@ -229,9 +230,13 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const float ninf = -__int_as_float(0x7f800000);
     constexpr int kbt = kTileN / gpb;    // key blocks per key tile (2 s)
     constexpr int kbc = 32 / gpb;        // key blocks per 32-column chunk
+    bool complete = true;
     for (int J = 0; J <= jmax; ++J) {
       // every lane waits; the warp leaves together if any lane gave up
-      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full, J & 1, abort, args.status))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.acc_full, J & 1, abort, args.status))) {
+        complete = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll 1
       for (int ch = 0; ch < 8; ++ch) {
@@ -259,6 +264,25 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       if (lane == 0) mbar_arrive(&sm.acc_empty[e]);
       if (J == jmax && writer)
         for (int j = (jmax + 1) * kbt; j < args.nb_max; ++j) srow[j] = ninf;
+    }
+    if (args.fuse_select && complete) {
+      // Select the rows this warp scored: the query blocks whose groups are
+      // this warp's 32 lanes (their scores were written by this warp's
+      // writer lanes; __syncwarp orders those stores for the whole warp).
+      // Every product of the CTA has completed (the last acc_full), so the
+      // operand stages are free: they hold each warp's keys and histogram.
+      __syncwarp();
+      const size_t key_bytes = (static_cast<size_t>(args.nb_max) * 4 + 15) & ~size_t(15);
+      uint8_t* scratch = sm.stage[0] + static_cast<size_t>(warp) * (key_bytes + 1024);
+      uint32_t* keys = reinterpret_cast<uint32_t*>(scratch);
+      int* hist = reinterpret_cast<int*>(scratch + key_bytes);
+      for (int rb = 0; rb < 32 / gpb; ++rb) {
+        const int ib = (I * kTileM + q4 * 32) / gpb + rb;  // query block (local)
+        if (ib >= nb) break;
+        const size_t r = static_cast<size_t>(h) * args.nbtot + batch.g0[seq] + ib;
+        warp_select_row(args.scores + r * static_cast<size_t>(args.nb_max), ib, args.budgets[r], args.sink,
+                        args.window, keys, hist, args.col_idx + args.row_ptr[r]);
+      }
     }
   }
 

@@ -19,6 +19,7 @@
 //    chosen indices in ascending order.  No host round trip; HBM-bound.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
+#include "stem_select_row.cuh"
 
 namespace stem {
 
@@ -51,12 +52,6 @@ __device__ __forceinline__ int block_inclusive_scan(int x, int* s_warp, int* tot
   if (total) *total = s_warp[kThreads / 32 - 1];
   __syncthreads();
   return res;
-}
-
-__device__ __forceinline__ uint32_t order_key(float f) {
-  if (f != f) f = -__int_as_float(0x7f800000);  // NaN ranks as -inf
-  const uint32_t u = __float_as_uint(f);
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
 }  // namespace

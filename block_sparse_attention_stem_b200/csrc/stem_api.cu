@@ -224,8 +224,11 @@ double sm_scale(const stem_params_t* p) {
 // ---------------------------------------------------------------- stages
 // Every run_* below handles the KV heads hk0 .. hk0 + nhk - 1 (and their query
 // heads) only, so a caller can work through a layer one KV-head group at a time.
+// With budgets / row_ptr / col_idx given (fused selection), the budgets must
+// already be complete: the scoring CTAs then also write the lists.
 stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk, float* scores,
-                        float* vbonus, int* status, cudaStream_t stream) {
+                        float* vbonus, int* status, cudaStream_t stream, const int32_t* budgets = nullptr,
+                        const int32_t* row_ptr = nullptr, int32_t* col_idx = nullptr) {
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads, s = p->stride;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
@@ -254,6 +257,12 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   a.scores = scores;
   a.status = status;
   a.hk0 = hk0;
+  a.fuse_select = budgets != nullptr;
+  a.sink = p->sink_blocks;
+  a.window = p->window_blocks;
+  a.budgets = budgets;
+  a.row_ptr = row_ptr;
+  a.col_idx = col_idx;
   // one CTA per (pair of query heads of a KV group, 128-group query tile)
   const int pairs = nhk * ((hq / hkv + 1) / 2);
   for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return pairs * ((si.nb + s - 1) / s); })) {
@@ -274,9 +283,16 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   return STEM_OK;
 }
 
+// The scoring kernel selects the rows it scored (no separate selection pass)
+// for per-head lists whose rows fit its scratch.
+bool fuse_selection(const stem_params_t* p, const Plan& pl) {
+  return p->list_mode == STEM_LIST_PER_HEAD && pl.pub.nb_max <= kFusedSelectMaxBlocks;
+}
+
 stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
                          bool with_budgets, const float* scores,
-                         int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, cudaStream_t stream) {
+                         int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, cudaStream_t stream,
+                         bool with_lists = true) {
   const int hq = qkv->num_q_heads;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
   const int G = hq / qkv->num_kv_heads;
@@ -291,6 +307,7 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
   // block) when the query heads of a group share their lists
   const int per_list = p->list_mode == STEM_LIST_PER_GROUP ? G : 1;
   for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * (G / per_list) * si.nb; })) {
+    if (!with_lists) break;
     stem_status_t st = cuda_status(launch_select(b, hq, hk0 * G, nhk * G, per_list, nbtot, nb_max, p->sink_blocks,
                                                  p->window_blocks, scores,
                                                  budgets, row_ptr, col_idx, stream));
@@ -379,6 +396,29 @@ stem_status_t stem_score(const stem_qkv_t* qkv, const stem_params_t* params, flo
   return run_score(qkv, params, pl, 0, qkv->num_kv_heads, scores, vb, static_cast<int*>(ws), s);
 }
 
+stem_status_t stem_score_select(const stem_qkv_t* qkv, const stem_params_t* params, float* scores, float* vbonus,
+                                int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
+                                stem_stream_t stream) {
+  Plan pl;
+  stem_status_t st = make_plan(qkv, params, &pl);
+  if (st != STEM_OK) return st;
+  if ((st = check_tensors(qkv)) != STEM_OK) return st;
+  if (!scores || !budgets || !row_ptr || !ws || (!col_idx && pl.pub.nnz > 0)) return STEM_ERR_INVALID_ARG;
+  if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if ((st = clear_status(ws, s)) != STEM_OK) return st;
+  float* vb = vbonus ? vbonus : reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + pl.off_vbonus);
+  int* status = static_cast<int*>(ws);
+  const int hkv = qkv->num_kv_heads;
+  if (fuse_selection(params, pl)) {
+    if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s, false)) != STEM_OK)
+      return st;
+    return run_score(qkv, params, pl, 0, hkv, scores, vb, status, s, budgets, row_ptr, col_idx);
+  }
+  if ((st = run_score(qkv, params, pl, 0, hkv, scores, vb, status, s)) != STEM_OK) return st;
+  return run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s);
+}
+
 stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* params, const float* scores,
                           int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, void* ws, size_t ws_bytes,
                           stem_stream_t stream) {
@@ -457,8 +497,15 @@ stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, v
   int32_t* col_idx = col_idx_out ? col_idx_out : reinterpret_cast<int32_t*>(w + pl.off_colidx);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
   const int hkv = qkv->num_kv_heads;
-  if ((st = run_score(qkv, params, pl, 0, hkv, scores, vbonus, status, s)) != STEM_OK) return st;
-  if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
+  if (fuse_selection(params, pl)) {
+    // budgets first; the scoring CTAs then select the rows they scored
+    if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s, false)) != STEM_OK ||
+        (st = run_score(qkv, params, pl, 0, hkv, scores, vbonus, status, s, budgets, row_ptr, col_idx)) != STEM_OK)
+      return st;
+  } else {
+    if ((st = run_score(qkv, params, pl, 0, hkv, scores, vbonus, status, s)) != STEM_OK) return st;
+    if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
+  }
   return run_bsa(qkv, params, pl, 0, hkv, row_ptr, col_idx, out, lse, status, s);
 }
 
@@ -545,9 +592,21 @@ stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_params_t* para
     const int hk0 = g * per, nhk = (hk0 + per <= hkv) ? per : hkv - hk0;
     if (nhk <= 0) break;
     if ((e = cudaStreamWaitEvent(s, ev_in[g], 0)) != cudaSuccess) return fail(e);
-    if ((st = run_score(qkv, params, pl, hk0, nhk, scores, vbonus, status, s)) != STEM_OK ||
-        (st = run_select(qkv, params, pl, hk0, nhk, g == 0, scores, budgets, row_ptr, col_idx, s)) != STEM_OK ||
-        (st = run_bsa(qkv, params, pl, hk0, nhk, row_ptr, col_idx, out_dev, lse_dev, status, s)) != STEM_OK) {
+    const bool fused = fuse_selection(params, pl);
+    if (fused) {
+      // budgets (all heads) before the first group's scoring, which selects too
+      if ((g == 0 &&
+           (st = run_select(qkv, params, pl, hk0, nhk, true, scores, budgets, row_ptr, col_idx, s, false)) != STEM_OK) ||
+          (st = run_score(qkv, params, pl, hk0, nhk, scores, vbonus, status, s, budgets, row_ptr, col_idx)) != STEM_OK) {
+        release();
+        return st;
+      }
+    } else if ((st = run_score(qkv, params, pl, hk0, nhk, scores, vbonus, status, s)) != STEM_OK ||
+               (st = run_select(qkv, params, pl, hk0, nhk, g == 0, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) {
+      release();
+      return st;
+    }
+    if ((st = run_bsa(qkv, params, pl, hk0, nhk, row_ptr, col_idx, out_dev, lse_dev, status, s)) != STEM_OK) {
       release();
       return st;
     }

@@ -39,7 +39,17 @@ struct ScoreArgs {
   const float* vbonus;      // [Hkv][NBtot]
   float* scores;            // [Hq][NBtot][nb_max]
   int* status;
+  // fused selection: when set, every CTA also selects the rows it scored
+  // (budgets and row_ptr must be complete; nb_max <= kFusedSelectMaxBlocks)
+  int fuse_select;
+  int sink, window;
+  const int32_t* budgets;
+  const int32_t* row_ptr;
+  int32_t* col_idx;
 };
+// largest nb_max for which the scoring kernel can select its rows itself (the
+// per-warp selection scratch lives in the drained operand stages)
+constexpr int kFusedSelectMaxBlocks = 5888;
 
 struct BsaArgs {
   int hq, hkv, nbtot, total_tokens;

@@ -200,6 +200,16 @@ STEM_API stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* p
                           const float* scores, int32_t* budgets, int32_t* row_ptr,
                           int32_t* col_idx, void* ws, size_t ws_bytes, stem_stream_t stream);
 
+/* stem_score and stem_select in one pass: same arguments and outputs as the two
+ * calls (scores, vbonus, budgets, row_ptr, col_idx), results bit for bit equal.
+ * With per-head lists and nb_max <= 5888 each scoring CTA selects the rows it has
+ * just scored (the budgets run first), so the scores are read back from L2 and
+ * no separate selection pass runs; otherwise the two passes run in turn. */
+STEM_API stem_status_t stem_score_select(const stem_qkv_t* qkv, const stem_params_t* params,
+                                float* scores, float* vbonus,
+                                int32_t* budgets, int32_t* row_ptr, int32_t* col_idx,
+                                void* ws, size_t ws_bytes, stem_stream_t stream);
+
 /* Causal block-sparse attention over caller-given CSR lists [gist-zh §2.3 exact
  * softmax over the chosen blocks only; youleyou §3.1].
  *   For query token t of block i of row r: keys = union over j in
@@ -229,7 +239,8 @@ STEM_API stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_page
                                  void* out, float* lse,
                                  void* ws, size_t ws_bytes, stem_stream_t stream);
 
-/* score -> select -> attention on one stream with no host round trip.
+/* score -> select -> attention on one stream with no host round trip (the
+ * selection fused into the scoring pass as in stem_score_select).
  * row_ptr_out / col_idx_out may be NULL (the workspace then holds the lists);
  * ws_bytes >= plan.ws_prefill_bytes. */
 STEM_API stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params,

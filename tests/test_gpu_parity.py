@@ -101,6 +101,20 @@ def test_select_is_bit_exact_on_identical_fp32_scores(name):
     assert np.array_equal(gci.cpu().numpy(), oci)
 
 
+@pytest.mark.parametrize("name", list(CASES))
+def test_score_select_equals_score_then_select(name):
+    """The fused pass (scoring CTAs selecting their own rows) gives exactly the
+    two separate passes' scores and lists."""
+    c = get_case(name)
+    scores, vbonus, ws = b.stem_score(c.qkv, c.params)
+    gb, grp, gci, _ = b.stem_select(c.qkv, c.params, scores)
+    s2, gb2, grp2, gci2, ws2 = b.stem_score_select(c.qkv, c.params)
+    torch.cuda.synchronize()
+    assert b.stem_read_device_status(ws2) == 0
+    assert torch.equal(s2.view(torch.int32), scores.view(torch.int32))
+    assert torch.equal(gb2, gb) and torch.equal(grp2, grp) and torch.equal(gci2, gci)
+
+
 def test_select_ties_go_to_lowest_index():
     c = get_case("varlen")
     rng = np.random.default_rng(3)
