@@ -58,7 +58,8 @@ class StemPlan(ctypes.Structure):
                 ("nnz", ctypes.c_int64), ("nnz_per_head", ctypes.c_int64), ("scores_bytes", ctypes.c_size_t),
                 ("vbonus_bytes", ctypes.c_size_t), ("ws_bytes", ctypes.c_size_t),
                 ("ws_prefill_bytes", ctypes.c_size_t), ("attn_flops", ctypes.c_double),
-                ("dense_attn_flops", ctypes.c_double), ("score_flops", ctypes.c_double)]
+                ("dense_attn_flops", ctypes.c_double), ("score_flops", ctypes.c_double),
+                ("vwide_bytes", ctypes.c_size_t)]
 
 
 class StemError(RuntimeError):

@@ -21,19 +21,22 @@
 // With two S buffers, S_{h+1} is computed while the softmax of half h runs, so
 // the softmax does not wait for the tensor core in steady state.
 // The reference row max m moves (and O is rescaled in TMEM) only when a half
-// raises it past a threshold (2^8 bf16, 2^1 fp8), so P stays bounded and
+// raises it past a threshold (2^8), so P stays bounded and
 // rescales are rare; O and the row sum share that reference, so the result is
 // exact.  A rescale first waits for P_{h-1} V_{h-1} (S_h does not imply it).
 // Masking happens only on the diagonal block.
 //
-// fp8: a single e4m3 P carries three mantissa bits (up to 6% error per weight,
-// which rows with few keys cannot average out), so P*224 is split into
-// hi = e4m3(P*224) and lo = e4m3(remainder); two e4m3 MMAs accumulate hi.V and
-// lo.V into the same O, leaving P about eight significant bits.
+// fp8: Q K^T runs on e4m3 operands (kind::f8f6f4).  A single e4m3 P would
+// carry three mantissa bits (up to 6% error per weight, which rows with few
+// keys cannot average out), so P is kept in f16 and P V runs as an f16
+// product (kind::f16) against V widened to f16 beforehand (every e4m3 value is
+// an f16 value, so the widening is exact).  Two e4m3 products of a split P
+// would take the same tensor time as the one f16 product, and more
+// conversions per weight.
 //
 // P is written over S in place: chunk ch (keys 32ch..32ch+31 of the half)
-// goes to columns 16ch..16ch+15 of the S buffer (bf16 pairs, or 8 columns of
-// hi and 8 of lo for e4m3); the whole half is in registers by then.
+// goes to columns 16ch..16ch+15 of the S buffer (bf16 or f16 pairs); the whole
+// half is in registers by then.
 //
 // Warp roles (224 threads):
 //   warps 0-3  softmax + epilogue (TMEM lane quarters 0-3)
@@ -67,18 +70,19 @@ constexpr uint32_t kPolyMask = STEM_BSA_POLY_MASK;
 
 template <bool kFp8>
 struct BsaCfg {
-  static constexpr int kQBytes = kFp8 ? 16384 : 32768;    // one 128 x 128 Q block
-  static constexpr int kHalfBytes = kFp8 ? 8192 : 16384;  // 64 keys x 128 dims of K or V
-  static constexpr float kRescaleLog2 = kFp8 ? 1.f : 8.f;  // max growth before O is rescaled
-  static constexpr float kPScale = kFp8 ? 224.f : 1.f;     // P multiplier before rounding (e4m3: 2 * 224 = 448)
+  static constexpr int kQBytes = kFp8 ? 16384 : 32768;     // one 128 x 128 Q block
+  static constexpr int kKHalfBytes = kFp8 ? 8192 : 16384;  // 64 keys x 128 dims of K
+  static constexpr int kVHalfBytes = 16384;                // 64 keys x 128 dims of V (bf16 or f16)
+  static constexpr int kKSlabs = kFp8 ? 1 : 2;             // 128-byte head-dim slabs per K row
+  static constexpr float kRescaleLog2 = 8.f;               // max growth before O is rescaled
 };
 template struct BsaCfg<true>;
 
 template <bool kFp8>
 struct BsaSmem {
   uint8_t q[BsaCfg<kFp8>::kQBytes];                        // 1024-aligned
-  uint8_t k[2][BsaCfg<kFp8>::kHalfBytes];                  // per slot
-  uint8_t v[2][BsaCfg<kFp8>::kHalfBytes];
+  uint8_t k[2][BsaCfg<kFp8>::kKHalfBytes];                 // per slot
+  uint8_t v[2][BsaCfg<kFp8>::kVHalfBytes];
   uint64_t q_full;
   uint64_t k_full[2];  // per slot: K_h landed
   uint64_t v_full[2];  // per slot: V_h landed
@@ -169,10 +173,10 @@ __device__ void stage_list(const int32_t* __restrict__ col, const Tile& t, int32
 
 // p = exp2(s c - m) for one 32-key chunk of a row: packed scale-and-shift,
 // exp2 (MUFU, or for the pairs in kPoly the FMA-pipe polynomial), packed row
-// sums and bf16 packing.  w[k] holds keys 2k (low half) and 2k + 1.
-template <uint32_t kPoly>
-__device__ __forceinline__ void exp_chunk_bf16(const uint32_t* rr, float2 c2, float2 nm2, float2& ps0, float2& ps1,
-                                               uint32_t* w) {
+// sums and bf16 (or f16) packing.  w[k] holds keys 2k (low half) and 2k + 1.
+template <uint32_t kPoly, bool kF16>
+__device__ __forceinline__ void exp_chunk(const uint32_t* rr, float2 c2, float2 nm2, float2& ps0, float2& ps1,
+                                          uint32_t* w) {
 #pragma unroll
   for (int x = 0; x < 16; x += 2) {
     const float2 a = ffma2(make_float2(__uint_as_float(rr[2 * x]), __uint_as_float(rr[2 * x + 1])), c2, nm2);
@@ -181,8 +185,8 @@ __device__ __forceinline__ void exp_chunk_bf16(const uint32_t* rr, float2 c2, fl
     const float2 p23 = ((kPoly >> (x + 1)) & 1u) ? exp2_poly2(a2) : make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
     ps0 = fadd2(ps0, p01);
     ps1 = fadd2(ps1, p23);
-    w[x] = pack_bf16x2(p01.x, p01.y);
-    w[x + 1] = pack_bf16x2(p23.x, p23.y);
+    w[x] = kF16 ? f32x2_to_f16x2(p01.x, p01.y) : pack_bf16x2(p01.x, p01.y);
+    w[x + 1] = kF16 ? f32x2_to_f16x2(p23.x, p23.y) : pack_bf16x2(p23.x, p23.y);
   }
 }
 
@@ -192,7 +196,6 @@ template <bool kFp8>
 __global__ void __launch_bounds__(kBsaThreads, 2)
     bsa_kernel(const __grid_constant__ BsaMaps maps, const SeqBatch batch, const BsaArgs args) {
   using Cfg = BsaCfg<kFp8>;
-  constexpr int kSlabs = kFp8 ? 1 : 2;  // 128-byte head-dim slabs per row (bf16: dims 0-63 and 64-127)
   extern __shared__ uint8_t smem_raw[];
   BsaSmem<kFp8>& sm =
       *reinterpret_cast<BsaSmem<kFp8>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -249,13 +252,17 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
     // ------------------------------------------------------------ producers
     const bool is_v = warp == kVProducerWarp;
     if (lane == 0 && N > 0) {
-      const bool paged = args.page_table != nullptr;
+      // fp8 V is read from its packed f16 copy, which the widening pass
+      // gathered through the page table
+      const bool paged = args.page_table != nullptr && !(kFp8 && is_v);
       const CUtensorMap* m = paged ? (is_v ? &maps.v_pool : &maps.k_pool) : (is_v ? &maps.v[seq] : &maps.k[seq]);
+      const int slabs = is_v ? 2 : Cfg::kKSlabs;
+      const int half_bytes = is_v ? Cfg::kVHalfBytes : Cfg::kKHalfBytes;
       const int32_t* pages = paged ? args.page_table + static_cast<size_t>(batch.seq_id[seq]) * args.max_pages : nullptr;
       tma_prefetch_desc(m);
       if (!is_v) {
         mbar_arrive_expect_tx(&sm.q_full, Cfg::kQBytes);
-        for (int hh = 0; hh < kSlabs; ++hh)
+        for (int hh = 0; hh < Cfg::kKSlabs; ++hh)
           tma_load_3d(sm.q + hh * 16384, &maps.q[seq], &sm.q_full, hh * 64, tl.h, tl.i * kBlock);
       }
       const int H = 2 * N;
@@ -274,8 +281,8 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
         // reads zeros)
         int row = j * kBlock + (h & 1) * kHalf;
         if (paged) row = __ldg(pages + row / args.page_size) * args.page_size + row % args.page_size;
-        mbar_arrive_expect_tx(bar, Cfg::kHalfBytes);
-        for (int hh = 0; hh < kSlabs; ++hh) tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, row);
+        mbar_arrive_expect_tx(bar, half_bytes);
+        for (int hh = 0; hh < slabs; ++hh) tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, row);
         ++issued;
       }
       // every copy of this producer has landed before the CTA can exit (a
@@ -292,7 +299,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0 && N > 0) {
       const uint32_t idesc_s = make_idesc(kFp8 ? 0u : 1u, 0u, 128u, static_cast<uint32_t>(kHalf));
-      const uint32_t idesc_o = make_idesc(kFp8 ? 0u : 1u, 1u, 128u, 128u);
+      const uint32_t idesc_o = make_idesc(kFp8 ? 0u : 1u, 1u, 128u, 128u);  // kind::f16: f16 (0) or bf16 (1)
       const uint32_t sq = smem_u32(sm.q);
       const uint32_t o_tmem = tmem + 128;
       const int H = 2 * N;
@@ -321,19 +328,11 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
         tc_fence_after();
         const uint32_t sv = smem_u32(sm.v[h & 1]);
         const uint32_t p = tmem + kHalf * (h & 1);
-        if constexpr (kFp8) {
+        // kind::f16 for both: bf16 P and V, or f16 P and V (the fp8 path)
 #pragma unroll
-          for (int kk = 0; kk < 2; ++kk)        // 32 keys per step
-#pragma unroll
-            for (int part = 0; part < 2; ++part)  // hi at 16 kk, lo at 16 kk + 8
-              mma_f8_ts(o_tmem, p + kk * 16 + part * 8, make_sdesc_sw128(sv + kk * 4096, kHalf * 128, 1024), idesc_o,
-                        (h | part | kk) != 0);
-        } else {
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // 16 keys per step
-            mma_bf16_ts(o_tmem, p + kk * 8, make_sdesc_sw128(sv + kk * 2048, kHalf * 128, 1024), idesc_o,
-                        (h | kk) != 0);
-        }
+        for (int kk = 0; kk < 4; ++kk)  // 16 keys per step
+          mma_bf16_ts(o_tmem, p + kk * 8, make_sdesc_sw128(sv + kk * 2048, kHalf * 128, 1024), idesc_o,
+                      (h | kk) != 0);
         mma_commit(&sm.v_free[h & 1]);
         if (h == H - 1) mma_commit(&sm.o_done);
         return true;
@@ -437,39 +436,13 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
         float2 ps0 = make_float2(0.f, 0.f), ps1 = make_float2(0.f, 0.f);
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
-          if constexpr (kFp8) {
-            uint32_t whi[8], wlo[8];
-#pragma unroll
-            for (int x = 0; x < 8; ++x) {
-              const float2 a = ffma2(make_float2(__uint_as_float(rr[ch][4 * x]), __uint_as_float(rr[ch][4 * x + 1])),
-                                     c2, nm2);
-              const float2 a2 = ffma2(
-                  make_float2(__uint_as_float(rr[ch][4 * x + 2]), __uint_as_float(rr[ch][4 * x + 3])), c2, nm2);
-              const float2 p01 = make_float2(fast_exp2(a.x), fast_exp2(a.y));
-              const float2 p23 = make_float2(fast_exp2(a2.x), fast_exp2(a2.y));
-              ps0 = fadd2(ps0, p01);
-              ps1 = fadd2(ps1, p23);
-              const uint32_t x01 = f32x2_to_f16x2(p01.x * Cfg::kPScale, p01.y * Cfg::kPScale);
-              const uint32_t x23 = f32x2_to_f16x2(p23.x * Cfg::kPScale, p23.y * Cfg::kPScale);
-              const uint16_t h01 = f16x2_to_e4m3x2(x01), h23 = f16x2_to_e4m3x2(x23);
-              const uint16_t l01 = f16x2_to_e4m3x2(hsub2_u32(x01, e4m3x2_to_f16x2(h01)));
-              const uint16_t l23 = f16x2_to_e4m3x2(hsub2_u32(x23, e4m3x2_to_f16x2(h23)));
-              whi[x] = static_cast<uint32_t>(h01) | (static_cast<uint32_t>(h23) << 16);
-              wlo[x] = static_cast<uint32_t>(l01) | (static_cast<uint32_t>(l23) << 16);
-            }
-            // 32 keys -> 8 columns of hi at 16 ch and 8 columns of lo at 16 ch + 8
-            tmem_st8(s_tmem + 16 * ch, whi);
-            tmem_st8(s_tmem + 16 * ch + 8, wlo);
+          uint32_t w[16];
+          if (diag) {
+            exp_chunk<0u, kFp8>(rr[ch], c2, nm2, ps0, ps1, w);  // masked keys need an exact 0
           } else {
-            uint32_t w[16];
-            if (diag) {
-              exp_chunk_bf16<0u>(rr[ch], c2, nm2, ps0, ps1, w);  // masked keys need an exact 0
-            } else {
-              exp_chunk_bf16<kPolyMask>(rr[ch], c2, nm2, ps0, ps1, w);
-            }
-            // 32 keys -> 16 columns at 16 ch
-            tmem_st16(s_tmem + 16 * ch, w);
+            exp_chunk<kPolyMask, kFp8>(rr[ch], c2, nm2, ps0, ps1, w);
           }
+          tmem_st16(s_tmem + 16 * ch, w);  // 32 keys -> 16 columns at 16 ch
         }
         l += (ps0.x + ps0.y) + (ps1.x + ps1.y);
         tmem_st_wait();
@@ -486,7 +459,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
       if (have_o) tc_fence_after();
       const bool store = t_row < L;
       float inv = (l > 0.f) ? 1.f / l : 0.f;
-      if constexpr (kFp8) inv *= args.v_scale[tl.hk] * (1.f / Cfg::kPScale);
+      if constexpr (kFp8) inv *= args.v_scale[tl.hk];
       uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) +
                                             (tok * args.hq + tl.h) * static_cast<size_t>(kHeadDim) * 2);
 #pragma unroll

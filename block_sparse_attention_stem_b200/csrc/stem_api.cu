@@ -33,7 +33,7 @@ struct SeqInfo {
 struct Plan {
   stem_plan_t pub;
   std::vector<SeqInfo> seqs;  // non-empty sequences, longest first
-  size_t off_vbonus, off_scores, off_budgets, off_rowptr, off_colidx;
+  size_t off_vbonus, off_vwide, off_scores, off_budgets, off_rowptr, off_colidx;
 };
 
 stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
@@ -106,8 +106,13 @@ stem_status_t make_plan(const stem_qkv_t* qkv, const stem_params_t* p, Plan* out
   pub.nnz_per_head = nnz_h;
   pub.scores_bytes = static_cast<size_t>(rows) * nb_max * sizeof(float);
   pub.vbonus_bytes = static_cast<size_t>(hkv) * nbtot * sizeof(float);
+  // fp8: the attention kernel reads V widened to f16 [T, Hkv, d]
+  pub.vwide_bytes = qkv->dtype == STEM_FP8_E4M3
+                        ? static_cast<size_t>(qkv->total_tokens) * hkv * kHeadDim * sizeof(uint16_t)
+                        : 0;
   pl.off_vbonus = kStatusBytes;
-  pub.ws_bytes = pl.off_vbonus + align256(pub.vbonus_bytes);
+  pl.off_vwide = pl.off_vbonus + align256(pub.vbonus_bytes);
+  pub.ws_bytes = pl.off_vwide + align256(pub.vwide_bytes);
   pl.off_scores = pub.ws_bytes;
   pl.off_budgets = pl.off_scores + align256(pub.scores_bytes);
   pl.off_rowptr = pl.off_budgets + align256(static_cast<size_t>(rows) * 4);
@@ -316,11 +321,25 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
   return STEM_OK;
 }
 
+// ws: the call's workspace (status word first, the widened V at off_vwide).
 stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
-                      const int32_t* row_ptr, const int32_t* col_idx, void* out, float* lse, int* status,
+                      const int32_t* row_ptr, const int32_t* col_idx, void* out, float* lse, void* ws,
                       cudaStream_t stream, const stem_paged_kv_t* paged = nullptr) {
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
+  int* status = static_cast<int*>(ws);
+  uint16_t* v16 = reinterpret_cast<uint16_t*>(static_cast<uint8_t*>(ws) + pl.off_vwide);
+  if (fp8) {
+    // V of these KV heads widened to f16, packed (gathered through the page
+    // table for paged K/V)
+    stem_status_t st = cuda_status(
+        paged ? launch_vwiden(paged->v_pages, v16, qkv->total_tokens, hkv, hk0, nhk, qkv->cu_seqlens,
+                              qkv->num_seqs, paged->page_table, paged->page_size, paged->num_pages,
+                              paged->max_pages_per_seq, stream)
+              : launch_vwiden(qkv->v, v16, qkv->total_tokens, hkv, hk0, nhk, nullptr, qkv->num_seqs, nullptr, 0,
+                              0, 0, stream));
+    if (st != STEM_OK) return st;
+  }
   BsaArgs a{};
   a.hq = hq;
   a.hkv = hkv;
@@ -343,7 +362,7 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
     // the page pool as one token sequence of pages * page_size rows
     const int pool = paged->num_pages * paged->page_size;
     if (!encode_seq_map(&maps.k_pool, paged->k_pages, fp8, hkv, 0, pool, kBlock / 2, 1) ||
-        !encode_seq_map(&maps.v_pool, paged->v_pages, fp8, hkv, 0, pool, kBlock / 2, 1))
+        (!fp8 && !encode_seq_map(&maps.v_pool, paged->v_pages, false, hkv, 0, pool, kBlock / 2, 1)))
       return STEM_ERR_CUDA;
     a.page_table = paged->page_table;
     a.page_size = paged->page_size;
@@ -356,8 +375,12 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
       // Q in 128-token boxes; K and V in 64-token boxes (the attention
       // kernel moves half a key block per copy)
       if (!encode_seq_map(&maps.q[q], qkv->q, fp8, hq, b.tok0[q], b.len[q], kBlock, 1)) return STEM_ERR_CUDA;
-      if (!paged && (!encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1) ||
-                     !encode_seq_map(&maps.v[q], qkv->v, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1)))
+      if (!paged && !encode_seq_map(&maps.k[q], qkv->k, fp8, hkv, b.tok0[q], b.len[q], kBlock / 2, 1))
+        return STEM_ERR_CUDA;
+      // V: the widened f16 copy (fp8), or the bf16 input when not paged
+      if ((fp8 || !paged) &&
+          !encode_seq_map(&maps.v[q], fp8 ? static_cast<const void*>(v16) : qkv->v, false, hkv, b.tok0[q], b.len[q],
+                          kBlock / 2, 1))
         return STEM_ERR_CUDA;
     }
     stem_status_t st = cuda_status(launch_bsa(maps, b, a, fp8, stream));
@@ -444,7 +467,7 @@ stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params, c
   if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
-  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s);
+  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, ws, s);
 }
 
 stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_paged_kv_t* kv, const stem_params_t* params,
@@ -474,7 +497,7 @@ stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_paged_kv_t* k
   if (ws_bytes < pl.pub.ws_bytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if ((st = clear_status(ws, s)) != STEM_OK) return st;
-  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, static_cast<int*>(ws), s, kv);
+  return run_bsa(qkv, params, pl, 0, qkv->num_kv_heads, row_ptr, col_idx, out, lse, ws, s, kv);
 }
 
 stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, void* out, float* lse,
@@ -506,7 +529,7 @@ stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params, v
     if ((st = run_score(qkv, params, pl, 0, hkv, scores, vbonus, status, s)) != STEM_OK) return st;
     if ((st = run_select(qkv, params, pl, 0, hkv, true, scores, budgets, row_ptr, col_idx, s)) != STEM_OK) return st;
   }
-  return run_bsa(qkv, params, pl, 0, hkv, row_ptr, col_idx, out, lse, status, s);
+  return run_bsa(qkv, params, pl, 0, hkv, row_ptr, col_idx, out, lse, ws, s);
 }
 
 stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_params_t* params, const void* q_host,
@@ -606,7 +629,7 @@ stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_params_t* para
       release();
       return st;
     }
-    if ((st = run_bsa(qkv, params, pl, hk0, nhk, row_ptr, col_idx, out_dev, lse_dev, status, s)) != STEM_OK) {
+    if ((st = run_bsa(qkv, params, pl, hk0, nhk, row_ptr, col_idx, out_dev, lse_dev, ws, s)) != STEM_OK) {
       release();
       return st;
     }

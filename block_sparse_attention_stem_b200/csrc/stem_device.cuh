@@ -211,7 +211,8 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
 }
 
 // Instruction descriptor (kind::f16 / kind::f8f6f4): fp32 accumulator,
-// A/B format code `fmt` (bf16 = 1 for kind::f16, e4m3 = 0 for kind::f8f6f4),
+// A/B format code `fmt` (f16 = 0 or bf16 = 1 for kind::f16, e4m3 = 0 for
+// kind::f8f6f4),
 // A K-major, B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t b_mn_major, uint32_t M, uint32_t N) {
   return (1u << 4)              // D format: f32

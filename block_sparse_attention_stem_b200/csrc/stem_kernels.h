@@ -90,6 +90,11 @@ cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int gro
                           cudaStream_t stream);
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
                        cudaStream_t stream);
+// fp8 V widened to f16 rows [T, Hkv, d] for KV heads hk0 .. hk0 + nhk - 1, read
+// packed or (page_table non-null) through the page table.
+cudaError_t launch_vwiden(const void* v8, uint16_t* v16, int total_tokens, int hkv, int hk0, int nhk,
+                          const int32_t* cu_seqlens, int num_seqs, const int32_t* page_table, int page_size,
+                          int num_pages, int max_pages, cudaStream_t stream);
 
 size_t score_smem_bytes();
 size_t bsa_smem_bytes(bool fp8);

@@ -151,12 +151,15 @@ typedef struct {
   int64_t nnz_per_head;      /* nnz / Hq */
   size_t  scores_bytes;      /* bytes of the fp32 score matrix [Hq][NBtot][nb_max] */
   size_t  vbonus_bytes;      /* bytes of the fp32 bonus [Hkv][NBtot] */
-  size_t  ws_bytes;          /* workspace for stem_score / stem_select / stem_bsa_fwd */
+  size_t  ws_bytes;          /* workspace for stem_score / stem_select / stem_bsa_fwd
+                                (includes vwide_bytes) */
   size_t  ws_prefill_bytes;  /* workspace for stem_prefill (holds scores and the CSR) */
   double  attn_flops;        /* 4 d Hq * (sum over listed blocks of query-key pairs), causal
                                 pairs only on the diagonal block */
   double  dense_attn_flops;  /* the same with every causal block listed */
   double  score_flops;       /* 2 * s * d * Hq * (16 x 16 group pairs per causal block pair) */
+  size_t  vwide_bytes;       /* fp8: the workspace's f16 copy of V [T, Hkv, d] that the
+                                attention reads (T * Hkv * d * 2 bytes); 0 for bf16 */
 } stem_plan_t;
 
 /* Validate (qkv, params) and fill *out.  Host only; touches no device memory
@@ -218,8 +221,10 @@ STEM_API stem_status_t stem_score_select(const stem_qkv_t* qkv, const stem_param
  *   sigma = softmax_scale (or 1/sqrt(d)), times q_scale*k_scale for fp8.
  * out bf16 [T, Hq, d]; lse fp32 [Hq][T].  Lists must be strictly ascending with
  * 0 <= j <= i; a violating entry is skipped and STEM_ERR_BAD_BLOCKLIST recorded.
- * An empty row gives out = 0 and lse = -inf.  fp8: P*224 is split into two e4m3
- * terms (hi + lo) whose two P.V products accumulate into O. */
+ * An empty row gives out = 0 and lse = -inf.  fp8: Q K^T runs on the e4m3
+ * operands; P is kept in f16 and P.V runs as an f16 product against V widened
+ * to f16 in the workspace (exact: every e4m3 value is an f16 value), since an
+ * e4m3 P (three mantissa bits) would miss the fp8 output tolerance. */
 STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params,
                            const int32_t* row_ptr, const int32_t* col_idx,
                            void* out, float* lse,

@@ -69,6 +69,10 @@ def test_plan_nnz_matches_oracle_budgets(name):
     pairs = sum(math.ceil(L / 128) * (math.ceil(L / 128) + 1) // 2 for L in w.seqlens)
     assert pl.score_flops == pytest.approx(2 * s * 128 * w.num_q_heads * pairs * (128 // s) ** 2)
     assert 0 < pl.attn_flops <= pl.dense_attn_flops
+    # fp8: the workspace holds V widened to f16 [T, Hkv, d] for the attention
+    T = sum(w.seqlens)
+    assert pl.vwide_bytes == (T * w.num_kv_heads * 128 * 2 if w.dtype == "fp8" else 0)
+    assert pl.ws_bytes >= pl.vwide_bytes and pl.ws_prefill_bytes >= pl.ws_bytes
 
 
 def test_plan_density_of_the_128k_workload():
