@@ -51,6 +51,8 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="long128k")
+    ap.add_argument("--dtype", choices=["bf16", "fp8"], default=None,
+                    help="override the workload's arithmetic type (same shapes and distributions)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
@@ -194,6 +196,11 @@ def bsa_traffic_per_launch(workload: str):
         return None
 
 
+def bench_workload(I, args):
+    """The named workload, with its arithmetic type overridden by --dtype."""
+    return I.workload(args.workload, **({"dtype": args.dtype} if args.dtype else {}))
+
+
 def describe(w) -> dict:
     return {
         "workload": (f"{w.name}: {len(w.seqlens)} x {w.seqlens if len(w.seqlens) > 1 else w.seqlens[0]} tokens, "
@@ -287,7 +294,7 @@ def run_ours(args):
     from block_sparse_attention_stem_b200 import binding as b
     from block_sparse_attention_stem_b200 import inputs as I
 
-    w = I.workload(args.workload)
+    w = bench_workload(I, args)
     seed = w.seed + 1000 * rank  # independent layer per rank
     inp = I.make_inputs(w, seed=seed, device="cuda")
     torch.cuda.synchronize()
@@ -414,7 +421,7 @@ def run_ours(args):
     if w.dtype == "fp8":
         peak *= 2.0  # nominal fp8 : bf16 dense ratio
     achieved = pl.attn_flops / (bsa_ms * 1e-3) / 1e12
-    traffic = bsa_traffic_per_launch(w.name)
+    traffic = bsa_traffic_per_launch(w.name if w.dtype == I.workload(w.name).dtype else f"{w.name}:{w.dtype}")
     roofline = {"bound": "tensor", "kernel": "bsa_kernel", "achieved": round(achieved, 2), "peak": peak,
                 "unit": "TFLOP/s", "frac": round(achieved / peak, 4), "traffic": traffic,
                 "peak_source": f"{peak_kind} bf16_tflops_sustained" + (" x2 (fp8 nominal ratio)" if w.dtype == "fp8"
@@ -462,7 +469,7 @@ def run_reference(args):
     import torch
     from block_sparse_attention_stem_b200 import inputs as I
 
-    w = I.workload(args.workload)
+    w = bench_workload(I, args)
     inp = I.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     host = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
     per_step = max(2.0, min(args.cpu_seconds, 20.0))
