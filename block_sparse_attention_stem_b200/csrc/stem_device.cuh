@@ -112,9 +112,6 @@ __device__ __forceinline__ bool mbar_wait_quiesce(uint64_t* bar, uint32_t parity
 }
 
 // ---------------------------------------------------------------- fences
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
 __device__ __forceinline__ void tc_fence_before() {
   asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
 }
@@ -193,15 +190,6 @@ __device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, ui
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
-__device__ __forceinline__ void mma_f8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t bdesc, uint32_t idesc,
-                                          uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
 
 // Arrive on `bar` once every tcgen05 operation this thread issued so far is done.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
@@ -210,10 +198,9 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
-// Instruction descriptor (kind::f16 / kind::f8f6f4): fp32 accumulator,
-// A/B format code `fmt` (f16 = 0 or bf16 = 1 for kind::f16, e4m3 = 0 for
-// kind::f8f6f4),
-// A K-major, B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
+// Instruction descriptor (kind::f16 / kind::f8f6f4): fp32 accumulator, A/B
+// format code `fmt` (f16 = 0 or bf16 = 1 for kind::f16; e4m3 = 0 for
+// kind::f8f6f4), A K-major, B K-major (b_mn_major = 0) or MN-major (1), shape M x N.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t fmt, uint32_t b_mn_major, uint32_t M, uint32_t N) {
   return (1u << 4)              // D format: f32
          | (fmt << 7)           // A format
@@ -274,29 +261,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
       "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
-  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"r"(taddr), "r"(r[0]),
-               "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-               : "memory");
-}
 __device__ __forceinline__ void tmem_st_wait() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
-
-// Per-warpgroup register budget change (all four warps of a warpgroup execute
-// the same one).  The increases of some warpgroups must be covered by the
-// decreases of others within the CTA's launch allocation, or .inc waits.
-template <uint32_t kRegs>
-__device__ __forceinline__ void warpgroup_regs_dec() {
-  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-template <uint32_t kRegs>
-__device__ __forceinline__ void warpgroup_regs_inc() {
-  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
-}
-
-// Named barrier over `nthreads` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // max of three floats in one instruction (sm_100).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
@@ -364,22 +329,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
-// Two floats -> two e4m3 bytes (lo in the low byte), saturating to +-448.
-__device__ __forceinline__ uint16_t pack_e4m3x2(float lo, float hi) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-
-// f32 pair -> f16x2 (lo in the low half); f16x2 <-> two e4m3 bytes.
+// f32 pair -> f16x2 (lo in the low half); two e4m3 bytes -> f16x2 (exact).
 __device__ __forceinline__ uint32_t f32x2_to_f16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
-  return r;
-}
-__device__ __forceinline__ uint16_t f16x2_to_e4m3x2(uint32_t h2) {
-  uint16_t r;
-  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(h2));
   return r;
 }
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
@@ -387,23 +340,9 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint16_t v) {
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(v));
   return r;
 }
-__device__ __forceinline__ uint32_t hsub2_u32(uint32_t a, uint32_t b) {
-  uint32_t r;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
-  return r;
-}
-
-// Two e4m3 bytes (lo in the low byte) -> their exact values as float2.
-__device__ __forceinline__ float2 unpack_e4m3x2(uint16_t v) {
-  uint32_t h2;
-  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
-  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
-}
 
 __device__ __forceinline__ int warp_id() { return static_cast<int>(threadIdx.x >> 5); }
 __device__ __forceinline__ int lane_id() { return static_cast<int>(threadIdx.x & 31); }
-
-__device__ __forceinline__ bool elect_one_lane() { return lane_id() == 0; }
 
 }  // namespace stem
 
