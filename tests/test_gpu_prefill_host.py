@@ -26,6 +26,11 @@ CASES = {
     "more_kv_heads_than_groups": W([640, 1024], 16, 16, seed=32),  # 16 KV heads -> 8 groups of 2
     "fp8_varlen": W([640, 2048, 77], 4, 2, dtype="fp8", seed=33),
     "qwen32k": I.workload("qwen32k"),
+    "one_kv_head": W([1000, 300], 4, 1, seed=34),  # a single group
+    "one_kv_head_odd_group": W([1500], 3, 1, seed=35),
+    "mha": W([700], 2, 2, seed=38),  # one query head per KV head
+    "std_bonus": W([1000, 128, 2088], 8, 2, seed=36, bonus_mode=1),  # per-KV-head z-score per group
+    "group_lists": W([1000, 2088], 8, 2, seed=37, list_mode=1),  # the separate selection pass
 }
 
 
