@@ -368,9 +368,13 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
     a.page_size = paged->page_size;
     a.max_pages = paged->max_pages_per_seq;
   }
-  // one CTA per CSR row (query head, query block)
+  // one CTA per CSR row (query head, query block), or, with lists shared by
+  // the query heads of a group, per (query block, pair of query heads)
   const int G = hq / hkv;
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return nhk * G * si.nb; })) {
+  const bool pairs = p->list_mode == STEM_LIST_PER_GROUP && G >= 2;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) {
+         return pairs ? nhk * ((G + 1) / 2) * si.nb : nhk * G * si.nb;
+       })) {
     for (int q = 0; q < b.n; ++q) {
       // Q in 128-token boxes; K and V in 64-token boxes (the attention
       // kernel moves half a key block per copy)
@@ -383,7 +387,8 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
                           kBlock / 2, 1))
         return STEM_ERR_CUDA;
     }
-    stem_status_t st = cuda_status(launch_bsa(maps, b, a, fp8, stream));
+    stem_status_t st =
+        cuda_status(pairs ? launch_bsa_pair(maps, b, a, fp8, stream) : launch_bsa(maps, b, a, fp8, stream));
     if (st != STEM_OK) return st;
   }
   return STEM_OK;

@@ -90,6 +90,11 @@ cudaError_t launch_select(const SeqBatch& batch, int hq, int h0, int nh, int gro
                           cudaStream_t stream);
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
                        cudaStream_t stream);
+// Rows whose lists are shared by the query heads of a KV group: one CTA per
+// (query block, pair of query heads), K and V staged once for the pair
+// (batch items: nhk * ceil(G / 2) * nb per sequence).
+cudaError_t launch_bsa_pair(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
+                            cudaStream_t stream);
 // fp8 V widened to f16 rows [T, Hkv, d] for KV heads hk0 .. hk0 + nhk - 1, read
 // packed or (page_table non-null) through the page table.
 cudaError_t launch_vwiden(const void* v8, uint16_t* v16, int total_tokens, int hkv, int hk0, int nhk,

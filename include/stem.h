@@ -224,7 +224,13 @@ STEM_API stem_status_t stem_score_select(const stem_qkv_t* qkv, const stem_param
  * An empty row gives out = 0 and lse = -inf.  fp8: Q K^T runs on the e4m3
  * operands; P is kept in f16 and P.V runs as an f16 product against V widened
  * to f16 in the workspace (exact: every e4m3 value is an f16 value), since an
- * e4m3 P (three mantissa bits) would miss the fp8 output tolerance. */
+ * e4m3 P (three mantissa bits) would miss the fp8 output tolerance.
+ * params->list_mode = STEM_LIST_PER_GROUP declares that the rows of the query
+ * heads of each KV group are identical (as stem_select writes them): each CTA
+ * then computes two query heads of one query block and stages each K/V tile
+ * once for both.  Rows of a pair that differ are reported as
+ * STEM_ERR_BAD_BLOCKLIST (the second head is then computed on the first
+ * head's list). */
 STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* params,
                            const int32_t* row_ptr, const int32_t* col_idx,
                            void* out, float* lse,

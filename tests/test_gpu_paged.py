@@ -52,6 +52,7 @@ CASES = {
     "varlen_page64": (W([1000, 128, 2088], 8, 2), 64),
     "gqa_page128": (W([1500, 700], 6, 2, seed=51), 128),
     "fp8_page256": (W([640, 2048, 77], 4, 2, dtype="fp8", seed=52), 256),
+    "shared_lists_page64": (W([1000, 128, 2088], 8, 2, seed=53, list_mode=1), 64),  # two heads per CTA
 }
 
 

@@ -48,6 +48,7 @@ CASES = {
     # one block list per KV head (max over its query heads), shared by the group
     "group_lists": W([1000, 128, 2088], 8, 2, seed=21, list_mode=1),
     "group_lists_odd_group": W([1500, 700], 6, 2, seed=22, list_mode=1, keep_ratio=0.25),
+    "group_lists_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=23, list_mode=1),
 }
 
 
@@ -194,3 +195,35 @@ def test_results_are_deterministic():
     z = b.stem_prefill(c.qkv, c.params)
     for x, y in zip(a[:4], z[:4]):
         assert torch.equal(x, y)
+
+
+@pytest.mark.parametrize("name", ["group_lists", "group_lists_odd_group", "group_lists_fp8"])
+def test_shared_list_pairs_equal_the_one_row_kernel(name):
+    """With shared lists the attention runs two query heads per CTA on one
+    staged K/V stream; per row it is the same arithmetic as one row per CTA."""
+    c = get_case(name)
+    _, _, rp, ci, _ = b.stem_prefill(c.qkv, c.params)
+    out_pair, lse_pair, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, ci)
+    assert b.stem_read_device_status(ws) == 0
+    per_row = b.make_params(**dict(c.w.params(), list_mode=0))
+    out_row, lse_row, ws2 = b.stem_bsa_fwd(c.qkv, per_row, rp, ci)
+    assert b.stem_read_device_status(ws2) == 0
+    assert torch.equal(out_pair.view(torch.int16), out_row.view(torch.int16))
+    assert torch.equal(lse_pair.view(torch.int32), lse_row.view(torch.int32))
+
+
+def test_shared_list_mode_reports_rows_that_differ():
+    c = get_case("group_lists")
+    _, _, rp, ci, _ = b.stem_prefill(c.qkv, c.params)
+    rp_h, ci_h = rp.cpu().numpy(), ci.cpu().numpy().copy()
+    seqs, nbtot = O.seq_blocks(c.cu)
+    # head 1 (second of the pair with head 0), block 12 of the third sequence
+    # (global block 9 + 12): swap one listed block for an unlisted causal one
+    r = 1 * nbtot + 9 + 12
+    row = ci_h[rp_h[r]:rp_h[r + 1]]
+    spare = [j for j in range(13) if j not in set(row.tolist())]
+    assert spare and len(row) >= 2
+    row[0] = spare[0]
+    ci_h[rp_h[r]:rp_h[r + 1]] = np.sort(row)
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, torch.from_numpy(ci_h).cuda())
+    assert b.stem_read_device_status(ws) == 7  # STEM_ERR_BAD_BLOCKLIST
