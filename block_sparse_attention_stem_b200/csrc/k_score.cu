@@ -238,30 +238,55 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         break;
       }
       tc_fence_after();
-#pragma unroll 1
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t r[32];
-        tmem_ld32(tmem + e * 256 + ch * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r);
+      // 1. pool each key block's gpb key groups in registers, straight out of
+      //    TMEM (groups past the end of the sequence excluded) ...
+      float pooled[kbt];
+#pragma unroll
+      for (int ch = 0; ch < 8; ch += 2) {
+        uint32_t r[2][32];  // two 32-column chunks per TMEM wait
+        tmem_ld32(tmem + e * 256 + ch * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r[0]);
+        tmem_ld32(tmem + e * 256 + (ch + 1) * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r[1]);
         tmem_ld_wait();
-        const int b0 = J * kTileN + ch * 32;  // first key group of the chunk
 #pragma unroll
-        for (int kb = 0; kb < kbc; ++kb) {
-          // max over the gpb key groups of this key block (groups past the end excluded) ...
-          float v = ninf;
+        for (int c2 = 0; c2 < 2; ++c2) {
+          const int b0 = J * kTileN + (ch + c2) * 32;  // first key group of the chunk
+          const bool inside = (b0 + 32) * s <= L;      // no group of the chunk past the end
 #pragma unroll
-          for (int cc = kb * gpb; cc < (kb + 1) * gpb; ++cc)
-            v = fmaxf(v, ((b0 + cc) * s < L) ? __uint_as_float(r[cc]) : ninf);
-          // ... and over the gpb query groups (consecutive lanes) of each query block
-          v = row_valid ? v : ninf;
+          for (int kb = 0; kb < kbc; ++kb) {
+            const int c0 = kb * gpb;
+            float v = ninf;
+            if (inside) {
 #pragma unroll
-          for (int off = gpb / 2; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-          const int j = J * kbt + ch * kbc + kb;
-          if (writer && j < args.nb_max) srow[j] = (j <= i) ? fmaf(v, scale, 0.f) + bonus[j] : ninf;
+              for (int cc = c0; cc < c0 + gpb; cc += 2)
+                v = fmax3(v, __uint_as_float(r[c2][cc]), __uint_as_float(r[c2][cc + 1]));
+            } else {
+#pragma unroll
+              for (int cc = c0; cc < c0 + gpb; cc += 2)
+                v = fmax3(v, ((b0 + cc) * s < L) ? __uint_as_float(r[c2][cc]) : ninf,
+                          ((b0 + cc + 1) * s < L) ? __uint_as_float(r[c2][cc + 1]) : ninf);
+            }
+            pooled[(ch + c2) * kbc + kb] = v;
+          }
         }
       }
+      // ... then hand the accumulator back: the next tile's products on this
+      // head can start while the rest of the epilogue runs
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.acc_empty[e]);
+      // 2. the max over the gpb query groups (consecutive lanes) of each query
+      //    block, scale, bonus (lane k holds the tile's k-th key block's), store
+      const int jl = J * kbt + lane;
+      const float bl = (lane < kbt && jl < nb) ? bonus[jl] : 0.f;
+#pragma unroll 1
+      for (int k = 0; k < kbt; ++k) {
+        float v = row_valid ? pooled[k] : ninf;
+#pragma unroll
+        for (int off = gpb / 2; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+        const float bk = __shfl_sync(0xffffffffu, bl, k);
+        const int j = J * kbt + k;
+        if (writer && j < args.nb_max) srow[j] = (j <= i) ? fmaf(v, scale, 0.f) + bk : ninf;
+      }
       if (J == jmax && writer)
         for (int j = (jmax + 1) * kbt; j < args.nb_max; ++j) srow[j] = ninf;
     }
