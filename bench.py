@@ -617,56 +617,65 @@ def run_quality(args):
     mean over rows of exp(lse_sparse - lse_dense).  Compares the output-aware
     metric (beta = 0.2) with the routing score alone (beta = 0), and the
     position-decay budget (mu = 0.7) with a uniform one (mu = 1) at the same
-    kept-block count.  Synthetic inputs: a check of the method's direction, not
-    an accuracy benchmark."""
+    kept-block count, on two input structures: i.i.d. Q and K (attention close
+    to uniform) and the block-topic structure of the input generator
+    (attention concentrated on the blocks of the query's topic, block-varying
+    value magnitudes).  Synthetic inputs: a check of the method's direction,
+    not an accuracy benchmark."""
     import torch
     from block_sparse_attention_stem_b200 import binding as b
     from block_sparse_attention_stem_b200 import inputs as I
-    w0 = I.workload("qwen32k")
-    inp = I.make_inputs(w0, device="cuda")
-    cu = w0.cu_seqlens()
-    qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], cu, cu_seqlens_dev=inp["cu_seqlens"])
-    nb = math.ceil(w0.seqlens[0] / 128)
-    hq = w0.num_q_heads
-    # dense reference: every causal block listed
-    counts = torch.arange(1, nb + 1, dtype=torch.int64).repeat(hq)
-    drp = torch.zeros(hq * nb + 1, dtype=torch.int32)
-    drp[1:] = torch.cumsum(counts, 0).to(torch.int32)
-    dci = torch.cat([torch.arange(c, dtype=torch.int32) for c in range(1, nb + 1)]).repeat(hq)
-    params0 = b.make_params(**w0.params())
-    o_dense, l_dense, _ = b.stem_bsa_fwd(qkv, params0, drp.cuda(), dci.cuda())
-    o_dense = o_dense.float()
-    nrm = torch.linalg.vector_norm(o_dense).item()
+    results = []
+    for structure in ("iid", "topics"):
+        w0 = I.workload("qwen32k", structure=structure)
+        inp = I.make_inputs(w0, device="cuda")
+        cu = w0.cu_seqlens()
+        qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], cu, cu_seqlens_dev=inp["cu_seqlens"])
+        nb = math.ceil(w0.seqlens[0] / 128)
+        hq = w0.num_q_heads
+        # dense reference: every causal block listed
+        counts = torch.arange(1, nb + 1, dtype=torch.int64).repeat(hq)
+        drp = torch.zeros(hq * nb + 1, dtype=torch.int32)
+        drp[1:] = torch.cumsum(counts, 0).to(torch.int32)
+        dci = torch.cat([torch.arange(c, dtype=torch.int32) for c in range(1, nb + 1)]).repeat(hq)
+        params0 = b.make_params(**w0.params())
+        o_dense, l_dense, _ = b.stem_bsa_fwd(qkv, params0, drp.cuda(), dci.cuda())
+        o_dense = o_dense.float()
+        nrm = torch.linalg.vector_norm(o_dense).item()
 
-    def nnz_of(**kw):
-        return b.stem_plan(qkv, b.make_params(**dict(w0.params(), **kw))).nnz_per_head
+        def nnz_of(**kw):
+            return b.stem_plan(qkv, b.make_params(**dict(w0.params(), **kw))).nnz_per_head
 
-    target = nnz_of(mu=0.7, keep_ratio=w0.keep_ratio)
-    lo, hi = 0.01, 1.0  # uniform-budget keep ratio with the same kept-block count
-    for _ in range(40):
-        mid = 0.5 * (lo + hi)
-        lo, hi = (mid, hi) if nnz_of(mu=1.0, keep_ratio=mid) < target else (lo, mid)
-    rho_eq = hi
-    causal = nb * (nb + 1) // 2
-    points = []
-    for label, kw in (("stem: OAM beta 0.2, TPD mu 0.7", dict(beta=0.2, mu=0.7)),
-                      ("routing score only: beta 0, mu 0.7", dict(beta=0.0, mu=0.7)),
-                      ("OAM beta 0.2, uniform budget mu 1 (same kept blocks)", dict(beta=0.2, mu=1.0, keep_ratio=rho_eq)),
-                      ("routing score only, uniform budget", dict(beta=0.0, mu=1.0, keep_ratio=rho_eq)),
-                      ("standardized bonus beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, bonus_mode=1)),
-                      ("KV-group-shared lists, beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, list_mode=1))):
-        params = b.make_params(**dict(w0.params(), **kw))
-        out, lse, _, _, ws = b.stem_prefill(qkv, params, return_lists=False)
-        torch.cuda.synchronize()
-        assert b.stem_read_device_status(ws) == 0
-        err = torch.linalg.vector_norm(out.float() - o_dense).item() / nrm
-        mass = torch.exp(lse - l_dense).mean().item()
-        pl = b.stem_plan(qkv, params)
-        points.append(dict(selection=label, density=round(pl.nnz_per_head / causal, 4),
-                           rel_error_vs_dense=round(err, 5), softmax_mass_kept=round(mass, 5), **kw))
+        target = nnz_of(mu=0.7, keep_ratio=w0.keep_ratio)
+        lo, hi = 0.01, 1.0  # uniform-budget keep ratio with the same kept-block count
+        for _ in range(40):
+            mid = 0.5 * (lo + hi)
+            lo, hi = (mid, hi) if nnz_of(mu=1.0, keep_ratio=mid) < target else (lo, mid)
+        rho_eq = hi
+        causal = nb * (nb + 1) // 2
+        points = []
+        for label, kw in (("stem: OAM beta 0.2, TPD mu 0.7", dict(beta=0.2, mu=0.7)),
+                          ("routing score only: beta 0, mu 0.7", dict(beta=0.0, mu=0.7)),
+                          ("OAM beta 0.2, uniform budget mu 1 (same kept blocks)",
+                           dict(beta=0.2, mu=1.0, keep_ratio=rho_eq)),
+                          ("routing score only, uniform budget", dict(beta=0.0, mu=1.0, keep_ratio=rho_eq)),
+                          ("standardized bonus beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, bonus_mode=1)),
+                          ("KV-group-shared lists, beta 0.2, mu 0.7", dict(beta=0.2, mu=0.7, list_mode=1))):
+            params = b.make_params(**dict(w0.params(), **kw))
+            out, lse, _, _, ws = b.stem_prefill(qkv, params, return_lists=False)
+            torch.cuda.synchronize()
+            assert b.stem_read_device_status(ws) == 0
+            err = torch.linalg.vector_norm(out.float() - o_dense).item() / nrm
+            mass = torch.exp(lse - l_dense).mean().item()
+            pl = b.stem_plan(qkv, params)
+            points.append(dict(selection=label, density=round(pl.nnz_per_head / causal, 4),
+                               rel_error_vs_dense=round(err, 5), softmax_mass_kept=round(mass, 5), **kw))
+        results.append({"inputs": structure, "points": points})
+        del inp, qkv, o_dense, l_dense
+        torch.cuda.empty_cache()
     res = {"metric": "attention reconstruction vs dense (32K, synthetic)", "unit": "relative Frobenius error",
-           "higher_is_better": False, "points": points, "config": describe(w0), "dtype": "bf16",
-           "data": "synthetic (seeded, device RNG)"}
+           "higher_is_better": False, "results": results, "config": describe(I.workload("qwen32k")),
+           "dtype": "bf16", "data": "synthetic (seeded, device RNG)"}
     print(json.dumps(res), flush=True)
 
 

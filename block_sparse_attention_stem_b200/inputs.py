@@ -20,6 +20,15 @@ Workloads (head_dim 128, 128-token blocks, stride 8 unless stated):
 
 Value rows are N(0,1) vectors scaled by exp(z), z ~ N(0, 0.5^2), so their norms
 are log-normal with sigma 0.5.  Q and K entries are N(0,1).
+
+``structure="topics"`` (used by the reconstruction-quality measurement) adds,
+after the draws above, a block-level topic structure under which attention is
+concentrated rather than near uniform: per KV head, 16 random unit topic
+directions; every 128-token block gets one topic per KV head; Q rows (of the
+group's query heads) and K rows get that direction times a, with
+a^2 / sqrt(d) = 6, so a key of the query's topic scores about +6 higher; and
+the V rows of each (KV head, block) are scaled by exp(0.8 z), z ~ N(0, 1), so
+blocks differ in value magnitude.
 """
 
 from __future__ import annotations
@@ -55,6 +64,7 @@ class Workload:
     budget_mode: int = 0
     bonus_mode: int = 0
     list_mode: int = 0
+    structure: str = "iid"  # "iid", or "topics" (block-level topic structure, see the module docstring)
 
     def params(self) -> dict:
         return dict(block_size=self.block_size, stride=self.stride, chunk_size=self.chunk_size,
@@ -113,7 +123,34 @@ def _draw(w: Workload, gen: torch.Generator):
             u = qm / qm.norm(dim=1, keepdim=True)
             n = min(4, e - o)
             k[o:o + n] += 3.0 * u[None]
+    if w.structure == "topics":
+        _add_topics(w, q, k, v, gen)
     return q, k, v
+
+
+def _add_topics(w: Workload, q, k, v, gen: torch.Generator, ntopics: int = 16, logit_gap: float = 6.0):
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    G = hq // hkv
+    dev = gen.device
+    a = (logit_gap * d ** 0.5) ** 0.5
+    cu = w.cu_seqlens()
+    for s in range(len(w.seqlens)):
+        o, e = cu[s], cu[s + 1]
+        L = e - o
+        if L <= 0:
+            continue
+        nb = (L + 127) // 128
+        dirs = torch.randn(hkv, ntopics, d, generator=gen, dtype=torch.float32, device=dev)
+        dirs /= dirs.norm(dim=2, keepdim=True)
+        topic = torch.randint(0, ntopics, (hkv, nb), generator=gen, device=dev)
+        vscale = torch.exp(0.8 * torch.randn(hkv, nb, generator=gen, dtype=torch.float32, device=dev))
+        blk = torch.arange(L, device=dev) // 128  # block of each token
+        for hk in range(hkv):
+            t_dir = dirs[hk][topic[hk][blk]]  # [L, d]
+            k[o:e, hk] += a * t_dir
+            q[o:e, hk * G:(hk + 1) * G] += a * t_dir[:, None, :]
+            v[o:e, hk] *= vscale[hk][blk][:, None]
 
 
 def _to_fp8(x: torch.Tensor):
