@@ -78,6 +78,13 @@ def _check_workload(w, samples):
         assert np.array_equal(last, np.broadcast_to(i_of_row, last.shape))  # the diagonal ends each row
     assert torch.isfinite(res["out"].float()).all()
     assert torch.isfinite(res["lse"]).all()
+    G = hq // w.num_kv_heads
+    if p.list_mode:  # shared lists: the rows of a group's query heads are identical
+        for hk in range(w.num_kv_heads):
+            r0 = rp[hk * G * nbtot:(hk * G + 1) * nbtot + 1]
+            for e in range(1, G):
+                re_ = rp[(hk * G + e) * nbtot:(hk * G + e + 1) * nbtot + 1]
+                assert np.array_equal(ci[r0[0]:r0[-1]], ci[re_[0]:re_[-1]])
     # --- sampled rows against the oracle
     ties = 0
     worst = [0.0, 0.0, 0.0]
@@ -90,18 +97,24 @@ def _check_workload(w, samples):
         r = h * nbtot + g0 + i
         ref_row = O.block_score_row(qh, kh, vh, i, p)
         gpu_row = res["scores"][h, g0 + i, :i + 1].cpu().numpy().astype(np.float64)
+        sel_row = ref_row
+        if p.list_mode:  # the list is selected on the group's elementwise max (NaN as -inf)
+            hk0 = (h // G) * G
+            rows = [ref_row if e == h else O.block_score_row(*_head_slices(inp, w, s, e), i, p)
+                    for e in range(hk0, hk0 + G)]
+            sel_row = np.max(np.where(np.isnan(rows), -np.inf, rows), axis=0)
         err = float(np.max(np.abs(gpu_row - ref_row) / np.maximum(1.0, np.abs(ref_row))))
         worst[0] = max(worst[0], err)
         assert err <= 1e-3, (s, h, i, err)
         G_list = ci[rp[r]:rp[r + 1]]
-        O_list = np.array(O.select_row(ref_row, i, int(bud[g0 + i]), p.sink_blocks, p.window_blocks))
+        O_list = np.array(O.select_row(sel_row, i, int(bud[g0 + i]), p.sink_blocks, p.window_blocks))
         if not np.array_equal(G_list, O_list):
             X = set(G_list.tolist()) - set(O_list.tolist())
             Y = set(O_list.tolist()) - set(G_list.tolist())
             assert len(X) == len(Y)
             for x in X:
                 for y in Y:
-                    assert abs(ref_row[x] - ref_row[y]) < TIE_REL * max(abs(ref_row[x]), abs(ref_row[y]))
+                    assert abs(sel_row[x] - sel_row[y]) < TIE_REL * max(abs(sel_row[x]), abs(sel_row[y]))
             ties += 1
         # attention of the row with the GPU's list
         rp1 = np.zeros(nb + 1, dtype=np.int64)
@@ -150,6 +163,13 @@ def test_fullsize_fp8_varlen_layers(layer):
 def test_fullsize_sweep64k_extremes(rho):
     w = I.workload("sweep64k", keep_ratio=rho)
     _check_workload(w, _samples(w, (7,), lambda nb: (2, nb - 1)))
+
+
+def test_fullsize_long128k_shared_lists():
+    """The bench workload with one list per KV group (list_mode 1): the
+    attention runs two query heads per CTA over K/V staged once for both."""
+    w = I.workload("long128k", list_mode=1)
+    _check_workload(w, _samples(w, (1, 18), lambda nb: (0, nb // 2, nb - 1)))
 
 
 def test_rows_longer_than_the_staged_list():
