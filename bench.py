@@ -231,7 +231,7 @@ def oracle_sample(w, host_inp, seconds: float, rows_hint=None):
     nb = math.ceil(L / 128)
     G = w.num_q_heads // w.num_kv_heads
     heads = sorted({h for h in (0, G, 2 * G + 1) if h < w.num_q_heads})
-    order = rows_hint or [(h, i) for i in list(range(nb - 1, -1, -max(1, nb // 16))) for h in heads]
+    order = rows_hint or [(h, i) for i in list(range(nb - 1, -1, -max(1, nb // 128))) for h in heads]
     cache = {}
 
     def head(h):
@@ -509,7 +509,7 @@ def run_reference(args):
     w = bench_workload(I, args)
     inp = I.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
     host = {k: (None if v is None else v.cpu()) for k, v in inp.items()}
-    per_step = max(2.0, min(args.cpu_seconds, 20.0))
+    per_step = max(1.0, min(args.cpu_seconds, 120.0 / max(1, args.steps)))  # the whole run stays near 2 min
     for _ in range(args.warmup):
         oracle_sample(w, host, per_step / 4)
     fl_tot, sec_tot, rows_tot = 0.0, 0.0, 0

@@ -72,13 +72,15 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
   const int ntile = (nb + s - 1) / s;  // query tiles of 128 groups = s blocks
-  // KV-head-major order (KV head, query tiles descending, head pairs of the
-  // group) so the CTAs in flight share one KV head's keys in L2.
+  // Query tiles descending across the launch's KV heads (query tile, KV head,
+  // head pair of the group): a CTA's work grows with its query tile, so the
+  // longest CTAs start first and the short ones fill the tail.
   const int G = args.hq / args.hkv;
   const int npair = (G + 1) / 2;
-  const int hk = args.hk0 + local / (npair * ntile);
-  const int rem = local % (npair * ntile);
-  const int I = ntile - 1 - rem / npair;  // longest rows first within a KV head
+  const int nhk = (batch.item0[seq + 1] - batch.item0[seq]) / (npair * ntile);  // KV heads in this launch
+  const int I = ntile - 1 - local / (nhk * npair);
+  const int rem = local % (nhk * npair);
+  const int hk = args.hk0 + rem / npair;
   const int h0 = hk * G + 2 * (rem % npair);
   const bool has1 = 2 * (rem % npair) + 1 < G;  // an odd group leaves the last pair one head
   const int halves = kFp8 ? 1 : 2;       // 64-element (bf16) or 128-element (fp8) K chunks per slot
