@@ -72,15 +72,29 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
   const int ntile = (nb + s - 1) / s;  // query tiles of 128 groups = s blocks
-  // Query tiles descending across the launch's KV heads (query tile, KV head,
-  // head pair of the group): a CTA's work grows with its query tile, so the
-  // longest CTAs start first and the short ones fill the tail.
+  // KV heads in groups of g; inside a group, query tiles descending (query
+  // tile, KV head, head pair of the group).  A CTA's work grows with its
+  // query tile.  When one KV head's CTAs outnumber the SMs, g = 1: the CTAs in
+  // flight stream one KV head's keys, which stay in L2, and the tail is short
+  // anyway.  Otherwise one KV head would leave the SMs unevenly loaded, and g
+  // is the largest divisor of the launch's KV heads whose keys fit in 64 MB,
+  // so each group starts its longest CTAs first and short ones fill the tail.
   const int G = args.hq / args.hkv;
   const int npair = (G + 1) / 2;
   const int nhk = (batch.item0[seq + 1] - batch.item0[seq]) / (npair * ntile);  // KV heads in this launch
-  const int I = ntile - 1 - local / (nhk * npair);
-  const int rem = local % (nhk * npair);
-  const int hk = args.hk0 + rem / npair;
+  int g = 1;
+  if (npair * ntile < args.num_sms) {
+    const size_t key_bytes = static_cast<size_t>(L) * 128 * (kFp8 ? 1 : 2);  // one KV head's keys
+    for (int c = nhk; c > 1; --c)
+      if (nhk % c == 0 && static_cast<size_t>(c) * key_bytes <= (size_t(64) << 20)) {
+        g = c;
+        break;
+      }
+  }
+  const int lg = local % (g * npair * ntile);
+  const int I = ntile - 1 - lg / (g * npair);
+  const int rem = lg % (g * npair);
+  const int hk = args.hk0 + (local / (g * npair * ntile)) * g + rem / npair;
   const int h0 = hk * G + 2 * (rem % npair);
   const bool has1 = 2 * (rem % npair) + 1 < G;  // an odd group leaves the last pair one head
   const int halves = kFp8 ? 1 : 2;       // 64-element (bf16) or 128-element (fp8) K chunks per slot
@@ -334,9 +348,14 @@ static cudaError_t launch_score_t(const ScoreMaps& maps, const SeqBatch& batch, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args, bool fp8,
+cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args_in, bool fp8,
                          cudaStream_t stream) {
   if (batch.item0[batch.n] == 0) return cudaSuccess;
+  ScoreArgs args = args_in;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e == cudaSuccess) e = cudaDeviceGetAttribute(&args.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
   if (args.stride == 8)
     return fp8 ? launch_score_t<true, 8>(maps, batch, args, stream) : launch_score_t<false, 8>(maps, batch, args, stream);
   if (args.stride == 4)

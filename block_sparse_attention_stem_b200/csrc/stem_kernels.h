@@ -33,6 +33,7 @@ struct BsaMaps {
 struct ScoreArgs {
   int hq, hkv, nbtot, nb_max, stride;
   int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
+  int num_sms;              // SMs of the device (the CTA order depends on it, never the results)
   float scale;              // 1 / (sqrt(d) s n)
   const float* q_scale;     // fp8 only
   const float* k_scale;
