@@ -42,6 +42,9 @@ CASES = {
     "varlen_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=16),
     "many_seqs": W([128 * (k % 5 + 1) + 8 * k for k in range(11)], 2, 1, seed=17),
     "gqa3_odd_group": W([1500, 700], 6, 2, seed=18),  # three query heads per KV head
+    # 36 KV heads of 2 MB of keys at 8K: the scoring CTAs run in two groups of
+    # 18 KV heads (the most that fit in 64 MB), query tiles descending in each
+    "mha36_grouped": W([8192], 36, 36, seed=24),
     # standardized value bonus (per-sequence, per-KV-head z-score of ln ||v||^2)
     "std_bonus_varlen": W([1000, 128, 2088], 8, 2, seed=19, bonus_mode=1),
     "std_bonus_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=20, bonus_mode=1),
