@@ -6,7 +6,8 @@
 //
 // One CTA per key block reads the block's 128 tokens x Hkv heads x 128 values
 // (256 KB bf16, contiguous in the packed [T, Hkv, d] layout) once with 16-byte
-// loads; 8 lanes cover one (token, head) row of 128 values.  HBM-bound.
+// loads; 16 (bf16) or 8 (fp8) lanes cover one (token, head) row of 128
+// values, and each thread keeps four rows' loads in flight.  HBM-bound.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -34,19 +35,32 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
   const int sub = threadIdx.x % kLanesPerRow;
   const int row_step = blockDim.x / kLanesPerRow;
   const uint8_t* base = v + (static_cast<size_t>(batch.tok0[s]) + t0) * hkv * kHeadDim * kElt;
-  for (int r0 = threadIdx.x / kLanesPerRow; r0 - static_cast<int>(threadIdx.x / kLanesPerRow) < rows;
-       r0 += row_step) {
-    float acc = 0.f;
-    const bool valid = r0 < rows;
-    if (valid) {
-      const size_t row = static_cast<size_t>(r0 / nhk) * hkv + hk0 + r0 % nhk;
-      const uint4 w = *reinterpret_cast<const uint4*>(base + row * kHeadDim * kElt + sub * 16);
-      const uint32_t u[4] = {w.x, w.y, w.z, w.w};
+  // four rows per thread in flight: their loads are issued before any of them
+  // is reduced (the trip count is uniform across a warp, so every lane takes
+  // part in the shuffles)
+  constexpr int kUnroll = 4;
+  const int first = threadIdx.x / kLanesPerRow;
+  for (int r0 = first; r0 - first < rows; r0 += kUnroll * row_step) {
+    uint4 w[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int r = r0 + u * row_step;
+      w[u] = make_uint4(0u, 0u, 0u, 0u);
+      if (r < rows) {
+        const size_t row = static_cast<size_t>(r / nhk) * hkv + hk0 + r % nhk;
+        w[u] = *reinterpret_cast<const uint4*>(base + row * kHeadDim * kElt + sub * 16);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int r = r0 + u * row_step;
+      const uint32_t q4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
+      float acc = 0.f;
       if constexpr (!kFp8) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float lo = __uint_as_float(u[q] << 16);
-          const float hi = __uint_as_float(u[q] & 0xFFFF0000u);
+          const float lo = __uint_as_float(q4[q] << 16);
+          const float hi = __uint_as_float(q4[q] & 0xFFFF0000u);
           acc = fmaf(lo, lo, acc);
           acc = fmaf(hi, hi, acc);
         }
@@ -55,7 +69,7 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
         for (int q = 0; q < 4; ++q) {
 #pragma unroll
           for (int b = 0; b < 4; b += 2) {
-            const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((u[q] >> (8 * b)) & 0xFFFFu);
+            const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((q4[q] >> (8 * b)) & 0xFFFFu);
             const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
             const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
             acc = fmaf(f.x, f.x, acc);
@@ -63,14 +77,14 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
           }
         }
       }
-    }
-    // reduce over the lanes of this row
+      // reduce over the lanes of this row
 #pragma unroll
-    for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (valid && sub == 0) {
-      const int h = r0 % nhk;
-      if constexpr (kFp8) acc *= v_scale[hk0 + h] * v_scale[hk0 + h];
-      atomicMax(&s_max[h], __float_as_uint(acc));
+      for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (r < rows && sub == 0) {
+        const int h = r % nhk;
+        if constexpr (kFp8) acc *= v_scale[hk0 + h] * v_scale[hk0 + h];
+        atomicMax(&s_max[h], __float_as_uint(acc));
+      }
     }
   }
   __syncthreads();
