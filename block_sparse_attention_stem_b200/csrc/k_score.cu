@@ -18,15 +18,17 @@
 // tile: a 64 KB stage (two 16 KB query slabs, one 32 KB key slab) feeds 1024
 // tensor cycles, where a single head's 48 KB stage fed 512.  The bytes moved
 // from L2 into shared memory per product are what bound this GEMM, so sharing
-// the key slab is what pays.  The epilogue warps (one warpgroup per head) read
-// their TMEM lane quarter, max-pool 16 columns in registers and 16 rows with
+// the key slab is what pays.  The epilogue warps (two warpgroups per head, one
+// per half of the accumulator's columns) read their TMEM lane quarter,
+// max-pool 16 columns in registers and 16 rows with
 // warp shuffles, scale, add the bonus and write one fp32 score per (query
 // block, key block); the next tile's products on a head wait only for that
 // head's epilogue.
 //
-// Warp roles (320 threads): warps 0-3 epilogue of the first head, warps 4-7 of
-// the second (TMEM lane quarter = warp % 4), warp 8 TMA producer, warp 9 TMEM
-// owner + MMA issuer.
+// Warp roles (576 threads): epilogue warps 0-15, warp w on head (w / 4) % 2,
+// TMEM lane quarter w % 4 and TMEM columns 128 (w / 8) .. +127 (two warps per
+// lane quarter, so a tile's accumulator is read back in half the time), warp
+// 16 TMA producer, warp 17 TMEM owner + MMA issuer.
 #include "stem_device.cuh"
 #include "stem_kernels.h"
 #include "stem_select_row.cuh"
@@ -35,9 +37,9 @@ namespace stem {
 
 namespace {
 
-constexpr int kScoreThreads = 320;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
+constexpr int kScoreThreads = 576;
+constexpr int kProducerWarp = 16;
+constexpr int kMmaWarp = 17;
 constexpr int kTileM = 128;            // query groups per tile (MMA M)
 constexpr int kTileN = 256;            // key groups per tile (MMA N)
 constexpr int kBytesA = kTileM * 128;  // one 128-B row per group and K-chunk, per head
@@ -111,7 +113,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       mbar_init(&sm.empty[i], 1);
     }
     mbar_init(&sm.acc_full, 1);
-    for (int i = 0; i < 2; ++i) mbar_init(&sm.acc_empty[i], 4);
+    for (int i = 0; i < 2; ++i) mbar_init(&sm.acc_empty[i], 8);
     mbar_init(&sm.drain, 1);
     sm.abort = 0;
     fence_mbar_init();
@@ -226,10 +228,12 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       mbar_wait_quiesce(&sm.drain, 0, args.status);
     }
     __syncwarp();
-  } else if (warp < 4 || has1) {
-    // epilogue: warpgroup e handles head h0 + e; thread owns TMEM lane (query
-    // group of the tile) `row`
-    const int e = warp >> 2;
+  } else if (((warp >> 2) & 1) == 0 || has1) {
+    // epilogue: warpgroups e and e + 2 handle head h0 + e, the first the key
+    // groups of TMEM columns 0-127 of each tile, the second columns 128-255;
+    // thread owns TMEM lane (query group of the tile) `row`
+    const int e = (warp >> 2) & 1;
+    const int half = warp >> 3;
     const int h = h0 + e;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
@@ -246,6 +250,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const float ninf = -__int_as_float(0x7f800000);
     constexpr int kbt = kTileN / gpb;    // key blocks per key tile (2 s)
     constexpr int kbc = 32 / gpb;        // key blocks per 32-column chunk
+    constexpr int kbh = kbt / 2;         // key blocks per half tile
     bool complete = true;
     for (int J = 0; J <= jmax; ++J) {
       // every lane waits; the warp leaves together if any lane gave up
@@ -256,16 +261,17 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       tc_fence_after();
       // 1. pool each key block's gpb key groups in registers, straight out of
       //    TMEM (groups past the end of the sequence excluded) ...
-      float pooled[kbt];
+      float pooled[kbh];
 #pragma unroll
-      for (int ch = 0; ch < 8; ch += 2) {
+      for (int ch = 0; ch < 4; ch += 2) {
         uint32_t r[2][32];  // two 32-column chunks per TMEM wait
-        tmem_ld32(tmem + e * 256 + ch * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r[0]);
-        tmem_ld32(tmem + e * 256 + (ch + 1) * 32 + (static_cast<uint32_t>(q4 * 32) << 16), r[1]);
+        const uint32_t col = e * 256 + half * 128 + ch * 32;
+        tmem_ld32(tmem + col + (static_cast<uint32_t>(q4 * 32) << 16), r[0]);
+        tmem_ld32(tmem + col + 32 + (static_cast<uint32_t>(q4 * 32) << 16), r[1]);
         tmem_ld_wait();
 #pragma unroll
         for (int c2 = 0; c2 < 2; ++c2) {
-          const int b0 = J * kTileN + (ch + c2) * 32;  // first key group of the chunk
+          const int b0 = J * kTileN + half * 128 + (ch + c2) * 32;  // first key group of the chunk
           const bool inside = (b0 + 32) * s <= L;      // no group of the chunk past the end
 #pragma unroll
           for (int kb = 0; kb < kbc; ++kb) {
@@ -295,23 +301,36 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       const int jl = J * kbt + lane;
       const float bl = (lane < kbt && jl < nb) ? bonus[jl] : 0.f;
 #pragma unroll 1
-      for (int k = 0; k < kbt; ++k) {
+      for (int k = 0; k < kbh; ++k) {
         float v = row_valid ? pooled[k] : ninf;
 #pragma unroll
         for (int off = gpb / 2; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
-        const float bk = __shfl_sync(0xffffffffu, bl, k);
-        const int j = J * kbt + k;
+        const float bk = __shfl_sync(0xffffffffu, bl, half * kbh + k);
+        const int j = J * kbt + half * kbh + k;
         if (writer && j < args.nb_max) srow[j] = (j <= i) ? fmaf(v, scale, 0.f) + bk : ninf;
       }
-      if (J == jmax && writer)
+      if (J == jmax && writer && half == 0)
         for (int j = (jmax + 1) * kbt; j < args.nb_max; ++j) srow[j] = ninf;
     }
-    if (args.fuse_select && complete) {
-      // Select the rows this warp scored: the query blocks whose groups are
-      // this warp's 32 lanes (their scores were written by this warp's
-      // writer lanes; __syncwarp orders those stores for the whole warp).
-      // Every product of the CTA has completed (the last acc_full), so the
-      // operand stages are free: they hold each warp's keys and histogram.
+    // the two warps of a lane quarter wrote the two halves of the same rows:
+    // both reach this barrier once, whatever ended their loop
+    switch (e * 4 + q4) {  // constant barrier ids 1-8, one per (head, lane quarter)
+      case 0: asm volatile("bar.sync 1, 64;" ::: "memory"); break;
+      case 1: asm volatile("bar.sync 2, 64;" ::: "memory"); break;
+      case 2: asm volatile("bar.sync 3, 64;" ::: "memory"); break;
+      case 3: asm volatile("bar.sync 4, 64;" ::: "memory"); break;
+      case 4: asm volatile("bar.sync 5, 64;" ::: "memory"); break;
+      case 5: asm volatile("bar.sync 6, 64;" ::: "memory"); break;
+      case 6: asm volatile("bar.sync 7, 64;" ::: "memory"); break;
+      default: asm volatile("bar.sync 8, 64;" ::: "memory"); break;
+    }
+    if (args.fuse_select && complete && half == 0) {
+      // Select the rows this lane quarter scored: the query blocks whose
+      // groups are its 32 lanes (their scores were written by the writer
+      // lanes of this warp and of its partner for the upper half of each tile;
+      // the barrier above orders those stores for both).  Every product of
+      // the CTA has completed (the last acc_full), so the operand stages are
+      // free: they hold each selecting warp's keys and histogram.
       __syncwarp();
       const size_t key_bytes = (static_cast<size_t>(args.nb_max) * 4 + 15) & ~size_t(15);
       uint8_t* scratch = sm.stage[0] + static_cast<size_t>(warp) * (key_bytes + 1024);
