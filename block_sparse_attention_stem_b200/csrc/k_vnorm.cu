@@ -7,7 +7,9 @@
 // One CTA per key block reads the block's 128 tokens x Hkv heads x 128 values
 // (256 KB bf16, contiguous in the packed [T, Hkv, d] layout) once with 16-byte
 // loads; 16 (bf16) or 8 (fp8) lanes cover one (token, head) row of 128
-// values, and each thread keeps four rows' loads in flight.  HBM-bound.
+// values, and each thread keeps four rows' loads in flight.  The arithmetic
+// per byte is small but not free (widening, packed FMAs, the row's lane
+// reduction), so it is kept to a few instructions per 16-byte load.
 #include <cuda_bf16.h>
 #include <cuda_fp8.h>
 
@@ -37,32 +39,41 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
   const uint8_t* base = v + (static_cast<size_t>(batch.tok0[s]) + t0) * hkv * kHeadDim * kElt;
   // four rows per thread in flight: their loads are issued before any of them
   // is reduced (the trip count is uniform across a warp, so every lane takes
-  // part in the shuffles)
+  // part in the shuffles).  Row r is (token r / nhk, head r % nhk); the pair
+  // is advanced by row_step without a division per row.
   constexpr int kUnroll = 4;
   const int first = threadIdx.x / kLanesPerRow;
+  const int q_step = row_step / nhk, r_step = row_step % nhk;
+  int quo = first / nhk, rem = first % nhk;
   for (int r0 = first; r0 - first < rows; r0 += kUnroll * row_step) {
     uint4 w[kUnroll];
+    int head[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int r = r0 + u * row_step;
+      head[u] = rem;
       w[u] = make_uint4(0u, 0u, 0u, 0u);
       if (r < rows) {
-        const size_t row = static_cast<size_t>(r / nhk) * hkv + hk0 + r % nhk;
+        const size_t row = static_cast<size_t>(quo) * hkv + hk0 + rem;
         w[u] = *reinterpret_cast<const uint4*>(base + row * kHeadDim * kElt + sub * 16);
+      }
+      quo += q_step;
+      rem += r_step;
+      if (rem >= nhk) {
+        rem -= nhk;
+        ++quo;
       }
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int r = r0 + u * row_step;
       const uint32_t q4[4] = {w[u].x, w[u].y, w[u].z, w[u].w};
-      float acc = 0.f;
+      float2 acc2 = make_float2(0.f, 0.f);  // even and odd elements, two FMAs per instruction
       if constexpr (!kFp8) {
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-          const float lo = __uint_as_float(q4[q] << 16);
-          const float hi = __uint_as_float(q4[q] & 0xFFFF0000u);
-          acc = fmaf(lo, lo, acc);
-          acc = fmaf(hi, hi, acc);
+          const float2 x = make_float2(__uint_as_float(q4[q] << 16), __uint_as_float(q4[q] & 0xFFFF0000u));
+          acc2 = ffma2(x, x, acc2);
         }
       } else {
 #pragma unroll
@@ -71,17 +82,17 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
           for (int b = 0; b < 4; b += 2) {
             const __nv_fp8x2_storage_t pair = static_cast<__nv_fp8x2_storage_t>((q4[q] >> (8 * b)) & 0xFFFFu);
             const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(pair, __NV_E4M3);
-            const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
-            acc = fmaf(f.x, f.x, acc);
-            acc = fmaf(f.y, f.y, acc);
+            const float2 x = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+            acc2 = ffma2(x, x, acc2);
           }
         }
       }
+      float acc = acc2.x + acc2.y;
       // reduce over the lanes of this row
 #pragma unroll
       for (int off = kLanesPerRow / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
       if (r < rows && sub == 0) {
-        const int h = r % nhk;
+        const int h = head[u];
         if constexpr (kFp8) acc *= v_scale[hk0 + h] * v_scale[hk0 + h];
         atomicMax(&s_max[h], __float_as_uint(acc));
       }
