@@ -186,13 +186,22 @@ def bsa_traffic_per_launch(workload: str):
     summary, valid only for the workload it was captured on and while the
     kernel source is the one that was profiled."""
     try:
-        rec = dict(line.split(None, 1) for line in open(TRAFFIC_FILE) if line.strip() and not line.startswith("#"))
+        rec, other = {}, {}
+        for line in open(TRAFFIC_FILE):
+            if not line.strip() or line.startswith("#"):
+                continue
+            key, val = line.split(None, 1)
+            if key == "bytes_per_launch":  # another workload: "bytes_per_launch <workload> <bytes>"
+                name, nbytes = val.split()
+                other[name] = float(nbytes)
+            else:
+                rec[key] = val
         src = open(os.path.join(ROOT, "block_sparse_attention_stem_b200", "csrc", "k_bsa.cu"), "rb").read()
         if rec.get("source_sha256", "").strip() != hashlib.sha256(src).hexdigest():
             return None
-        if rec.get("workload", "").strip() != workload:
-            return None
-        return float(rec["bytes_per_launch_full_workload"])
+        if rec.get("workload", "").strip() == workload:
+            return float(rec["bytes_per_launch_full_workload"])
+        return other.get(workload)
     except (OSError, ValueError, KeyError):
         return None
 
