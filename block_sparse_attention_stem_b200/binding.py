@@ -28,7 +28,7 @@ STEM_BF16, STEM_FP8_E4M3 = 0, 1
 EXPORTED = ("stem_plan", "stem_score", "stem_select", "stem_score_select", "stem_bsa_fwd", "stem_bsa_fwd_paged",
             "stem_prefill",
             "stem_prefill_host",
-            "stem_prefill_noalloc",
+            "stem_prefill_noalloc", "stem_noalloc_read_device_status",
             "stem_selftest_wait_timeout", "stem_read_device_status", "stem_status_string", "stem_version")
 
 
@@ -82,6 +82,7 @@ def _load() -> ctypes.CDLL:
     lib.stem_bsa_fwd_paged.argtypes = [P(StemQKV), P(StemPagedKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, sz, vp]
     lib.stem_prefill_noalloc.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp]
+    lib.stem_noalloc_read_device_status.argtypes = [vp, P(ctypes.c_int)]
     lib.stem_prefill_host.argtypes = [P(StemQKV), P(StemParams), vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.stem_selftest_wait_timeout.argtypes = [vp, vp]
     lib.stem_read_device_status.argtypes = [vp, vp, P(ctypes.c_int)]
@@ -89,7 +90,8 @@ def _load() -> ctypes.CDLL:
     lib.stem_status_string.restype = ctypes.c_char_p
     lib.stem_version.restype = ctypes.c_int32
     for name in ("stem_plan", "stem_score", "stem_select", "stem_bsa_fwd", "stem_prefill",
-                 "stem_prefill_noalloc", "stem_selftest_wait_timeout", "stem_read_device_status"):
+                 "stem_prefill_noalloc", "stem_noalloc_read_device_status", "stem_selftest_wait_timeout",
+                 "stem_read_device_status"):
         getattr(lib, name).restype = ctypes.c_int
     return lib
 
@@ -342,6 +344,15 @@ def stem_prefill_noalloc(qkv: QKV, params: StemParams, out=None, lse=None, row_p
     _check(LIB.stem_prefill_noalloc(ctypes.byref(qkv.desc), ctypes.byref(params), _ptr(out), _ptr(lse),
                                     _ptr(row_ptr), _ptr(col_idx), _stream(stream)), "stem_prefill_noalloc")
     return out, lse, row_ptr, (None if col_idx is None else col_idx[:pl.nnz])
+
+
+def stem_noalloc_read_device_status(stream=None) -> int:
+    """Status word of stem_prefill_noalloc's built-in workspace on the current
+    device (synchronises the stream)."""
+    out = ctypes.c_int(0)
+    _check(LIB.stem_noalloc_read_device_status(_stream(stream), ctypes.byref(out)),
+           "stem_noalloc_read_device_status")
+    return out.value
 
 
 def stem_selftest_wait_timeout(ws, stream=None):

@@ -4,6 +4,7 @@
 // the compute calls, no synchronisation.
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <cmath>
@@ -19,6 +20,17 @@ using namespace stem;
 namespace {
 
 constexpr size_t kStatusBytes = 256;
+
+// An NVTX range over one stage's host-side enqueue (scoring, selection,
+// attention), so a timeline profiler shows which launches belong to which
+// stage.  Header-only NVTX: without a profiler attached a push/pop is a few
+// nanoseconds and loads nothing.
+struct StageRange {
+  explicit StageRange(const char* name) { nvtxRangePushA(name); }
+  ~StageRange() { nvtxRangePop(); }
+  StageRange(const StageRange&) = delete;
+  StageRange& operator=(const StageRange&) = delete;
+};
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -234,6 +246,7 @@ double sm_scale(const stem_params_t* p) {
 stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk, float* scores,
                         float* vbonus, int* status, cudaStream_t stream, const int32_t* budgets = nullptr,
                         const int32_t* row_ptr = nullptr, int32_t* col_idx = nullptr) {
+  StageRange nvtx_range("stem: score");
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads, s = p->stride;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
@@ -298,6 +311,7 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
                          bool with_budgets, const float* scores,
                          int32_t* budgets, int32_t* row_ptr, int32_t* col_idx, cudaStream_t stream,
                          bool with_lists = true) {
+  StageRange nvtx_range("stem: select");
   const int hq = qkv->num_q_heads;
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
   const int G = hq / qkv->num_kv_heads;
@@ -325,6 +339,7 @@ stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Pl
 stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,
                       const int32_t* row_ptr, const int32_t* col_idx, void* out, float* lse, void* ws,
                       cudaStream_t stream, const stem_paged_kv_t* paged = nullptr) {
+  StageRange nvtx_range("stem: attention");
   const bool fp8 = qkv->dtype == STEM_FP8_E4M3;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
   int* status = static_cast<int*>(ws);

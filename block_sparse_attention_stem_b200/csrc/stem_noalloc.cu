@@ -19,8 +19,13 @@
 //    ordering between them) race and corrupt each other.  Serialise them.
 //  * The first call on each device looks up the array's device address (with
 //    that device current); make that first call before any stream capture.
-//  * Device-side errors are recorded in the built-in workspace; they are not
-//    reported by this call.
+//    The address is cached per device for the life of the process; it does
+//    not survive cudaDeviceReset.
+//  * `stream` must belong to the current device (STEM_ERR_INVALID_ARG
+//    otherwise), so the kernels never get another device's array.
+//  * Device-side errors (a bounded wait that ran out, a malformed list entry)
+//    are recorded in the built-in workspace's status word: read it with
+//    stem_noalloc_read_device_status after the call.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -54,7 +59,27 @@ void* static_ws_address() {
   return g_ws_addr[dev];
 }
 
+// STEM_OK when `stream` runs on the current device (the legacy and per-thread
+// default streams always do).
+stem_status_t check_stream_device(cudaStream_t stream) {
+  int cur = -1, sdev = -1;
+  if (cudaGetDevice(&cur) != cudaSuccess) return STEM_ERR_CUDA;
+  if (stream == nullptr || stream == cudaStreamLegacy || stream == cudaStreamPerThread) return STEM_OK;
+  if (cudaStreamGetDevice(stream, &sdev) != cudaSuccess) return STEM_ERR_INVALID_ARG;
+  return sdev == cur ? STEM_OK : STEM_ERR_INVALID_ARG;
+}
+
 }  // namespace
+
+extern "C" stem_status_t stem_noalloc_read_device_status(stem_stream_t stream, stem_status_t* out) {
+  if (!out) return STEM_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  stem_status_t st = check_stream_device(s);
+  if (st != STEM_OK) return st;
+  void* ws = static_ws_address();
+  if (ws == nullptr) return STEM_ERR_CUDA;
+  return stem_read_device_status(ws, stream, out);
+}
 
 extern "C" stem_status_t stem_prefill_noalloc(const stem_qkv_t* qkv, const stem_params_t* params, void* out,
                                               float* lse, int32_t* row_ptr_out, int32_t* col_idx_out,
@@ -63,6 +88,7 @@ extern "C" stem_status_t stem_prefill_noalloc(const stem_qkv_t* qkv, const stem_
   stem_status_t st = stem_plan(qkv, params, &pl);
   if (st != STEM_OK) return st;
   if (pl.ws_prefill_bytes > kStaticWorkspaceBytes) return STEM_ERR_WORKSPACE_TOO_SMALL;
+  if ((st = check_stream_device(reinterpret_cast<cudaStream_t>(stream))) != STEM_OK) return st;
   void* ws = static_ws_address();
   if (ws == nullptr) return STEM_ERR_CUDA;
   return stem_prefill(qkv, params, out, lse, row_ptr_out, col_idx_out, ws, kStaticWorkspaceBytes, stream);

@@ -16,10 +16,12 @@
 namespace stem {
 
 // Order-preserving 32-bit key of a float (larger float, larger key); NaN ranks
-// as -inf.
+// as -inf, and -0 and +0 get the same key (they compare equal as numbers, so
+// the lower block index wins between them, as for any other tie).
 __device__ __forceinline__ uint32_t order_key(float f) {
   if (f != f) f = -__int_as_float(0x7f800000);
-  const uint32_t u = __float_as_uint(f);
+  uint32_t u = __float_as_uint(f);
+  if (u == 0x80000000u) u = 0u;
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 

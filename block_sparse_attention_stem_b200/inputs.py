@@ -15,11 +15,13 @@ Workloads (head_dim 128, 128-token blocks, stride 8 unless stated):
 * ``long128k``   as qwen32k at 131072 tokens, 1 sink / 2 window blocks, seed 2.
 * ``sweep64k``   1 x 65536 tokens, 32 / 8 heads, mu 1.0, rho swept, seed 3.
 * ``fp8_varlen`` 4 packed sequences {8192, 16384, 40960, 98304}, e4m3 with
-                 per-head scale amax/448, rho 0.25, 36 layers with mu 1.0 for
+                 per-head scale amax/448 of N(0,1) data (Q, K and V alike; no
+                 value-norm scaling), rho 0.25, 36 layers with mu 1.0 for
                  layers 0-4 and 0.7 after, seed 4000 + layer.
 
-Value rows are N(0,1) vectors scaled by exp(z), z ~ N(0, 0.5^2), so their norms
-are log-normal with sigma 0.5.  Q and K entries are N(0,1).
+Value rows are N(0,1) vectors scaled by exp(z), z ~ N(0, sigma^2), so their
+norms are log-normal with sigma = ``v_norm_sigma`` (0.5; 0 leaves V at
+N(0,1)).  Q and K entries are N(0,1).
 
 ``structure="topics"`` (used by the reconstruction-quality measurement) adds,
 after the draws above, a block-level topic structure under which attention is
@@ -50,6 +52,7 @@ class Workload:
     dtype: str = "bf16"  # "bf16" or "fp8"
     seed: int = 0
     sink_boost: bool = False
+    v_norm_sigma: float = 0.5  # log-normal value-row norms; 0: plain N(0,1) rows
     # method parameters (values only)
     keep_ratio: float = 0.25
     mu: float = 0.7
@@ -96,7 +99,7 @@ def workload(name: str, **overrides) -> Workload:
                          mu=1.0, sink_blocks=4, window_blocks=4),
         "fp8_varlen": dict(seqlens=[8192, 16384, 40960, 98304], num_q_heads=32, num_kv_heads=8,
                            dtype="fp8", seed=4000, keep_ratio=0.25, mu=0.7, sink_blocks=4,
-                           window_blocks=4),
+                           window_blocks=4, v_norm_sigma=0.0),
     }[name]
     base.update(overrides)
     return Workload(name=name, **base)
@@ -113,7 +116,8 @@ def _draw(w: Workload, gen: torch.Generator):
     q = torch.randn(T, hq, d, generator=gen, dtype=torch.float32, device=dev)
     k = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32, device=dev)
     v = torch.randn(T, hkv, d, generator=gen, dtype=torch.float32, device=dev)
-    v *= torch.exp(0.5 * torch.randn(T, hkv, 1, generator=gen, dtype=torch.float32, device=dev))
+    if w.v_norm_sigma > 0:
+        v *= torch.exp(w.v_norm_sigma * torch.randn(T, hkv, 1, generator=gen, dtype=torch.float32, device=dev))
     if w.sink_boost:
         G = hq // hkv
         cu = w.cu_seqlens()

@@ -293,13 +293,25 @@ STEM_API stem_status_t stem_prefill_host(const stem_qkv_t* qkv, const stem_param
  *   All calls on a device share that array and it keeps the last call's
  *   contents: calls that may overlap on the GPU race; serialise them.
  *   The first call on each device looks up the array's address (with that
- *   device current); make it before any stream capture.
- *   Device-side errors go to the built-in workspace and are not reported here.
+ *   device current); make it before any stream capture.  The address is kept
+ *   for the life of the process and does not survive cudaDeviceReset.
+ *   `stream` must belong to the current device: STEM_ERR_INVALID_ARG if not.
+ *   Device-side errors go to the built-in workspace's status word: read them
+ *   with stem_noalloc_read_device_status.
  * Arguments, outputs and host-side errors are those of stem_prefill. */
 STEM_API stem_status_t stem_prefill_noalloc(const stem_qkv_t* qkv, const stem_params_t* params,
                                             void* out, float* lse,
                                             int32_t* row_ptr_out, int32_t* col_idx_out,
                                             stem_stream_t stream);
+
+/* The device status word of stem_prefill_noalloc's built-in workspace on the
+ * current device (no counterpart in the pages): synchronises `stream` (which
+ * must belong to the current device) and copies the word into *out, STEM_OK
+ * or the device-side error of the last call (STEM_ERR_TIMEOUT,
+ * STEM_ERR_BAD_BLOCKLIST).  Each stem_prefill_noalloc call clears it first.
+ * Returns STEM_ERR_INVALID_ARG for a NULL `out` or a stream of another device,
+ * STEM_ERR_CUDA if the copy fails. */
+STEM_API stem_status_t stem_noalloc_read_device_status(stem_stream_t stream, stem_status_t* out);
 
 /* Self-test of the device-side failure detection (no counterpart in the
  * pages).  Launches one kernel that waits, through the same bounded wait the

@@ -81,10 +81,51 @@ def compare_lists(rp_g, ci_g, rp_o, ci_o, ref_scores, cu, hq, sink, window, bloc
 
 def out_error(og, oo):
     """Output error scaled by max(1, |O_ref|): absolute where |O| <= 1 and
-    relative above.  The output is stored in bf16, whose own rounding is
-    2^-9 |O| (0.02 at |O| = 10), so a purely absolute 2e-2 bound cannot hold for
-    the large outputs that log-normal value norms produce."""
+    relative above (reported beside the checked figures below)."""
     return float((np.abs(og - oo) / np.maximum(1.0, np.abs(oo))).max())
+
+
+def bf16_rounding_interval(og):
+    """[lo, hi]: the reals that round (to nearest) to each bf16 value in og.
+    The bounds are the midpoints to the neighbouring bf16 values, taken from
+    the bit pattern (the encoding is sign-magnitude)."""
+    og = np.asarray(og, dtype=np.float64)
+    bits = (og.astype(np.float32).view(np.uint32) >> np.uint32(16)).astype(np.int64)
+    assert np.array_equal(((bits << 16).astype(np.uint32)).view(np.float32).astype(np.float64), og), \
+        "not bf16 values"
+    mag = bits & 0x7FFF
+    sign = np.where(bits & 0x8000, -1.0, 1.0)
+
+    def val(m):
+        return ((m.astype(np.uint32) << np.uint32(16)).view(np.float32)).astype(np.float64)
+
+    a = np.abs(og)
+    up = (a + val(np.minimum(mag + 1, 0x7F7F))) / 2
+    dn = np.where(mag > 0, (a + val(np.maximum(mag - 1, 0))) / 2, 0.0)
+    lo = np.where(sign > 0, dn, -up)
+    hi = np.where(sign > 0, up, -dn)
+    return lo, hi
+
+
+def out_error_abs(og, oo):
+    """Absolute output errors: (max |O_gpu - O_ref|, max |O_gpu - bf16(O_ref)|,
+    max distance from O_ref to the set of reals that round to O_gpu).  The
+    last one is what the max-abs bound is checked on: the GPU's output is a bf16
+    number, so the claim is that some value within the bound of the exact
+    result rounds to it — the part of |O_gpu - O_ref| that is the output's own
+    rounding (up to half a bf16 step, 2^-9 |O|) is not counted against the
+    arithmetic."""
+    og = np.asarray(og, dtype=np.float64)
+    oo = np.asarray(oo, dtype=np.float64)
+    raw = float(np.abs(og - oo).max()) if og.size else 0.0
+    rounded_ref = oo.astype(np.float32)
+    rounded_ref = (rounded_ref.view(np.uint32).astype(np.uint64) + 0x7FFF
+                   + ((rounded_ref.view(np.uint32) >> 16) & 1)) >> 16  # RNE to bf16
+    rounded_ref = ((rounded_ref.astype(np.uint32) << np.uint32(16)).view(np.float32)).astype(np.float64)
+    vs_rounded = float(np.abs(og - rounded_ref).max()) if og.size else 0.0
+    lo, hi = bf16_rounding_interval(og)
+    dist = np.maximum(np.maximum(lo - oo, oo - hi), 0.0)
+    return raw, vs_rounded, (float(dist.max()) if og.size else 0.0)
 
 
 def check_attention(out_g, lse_g, out_o, lse_o, dtype, rows_mask=None):
@@ -94,8 +135,12 @@ def check_attention(out_g, lse_g, out_o, lse_o, dtype, rows_mask=None):
         og, out_o = og[rows_mask], out_o[rows_mask]
         lg, lse_o = lg[:, rows_mask], lse_o[:, rows_mask]
     err = out_error(og, out_o)
+    raw, vs_rounded, beyond_rounding = out_error_abs(og, out_o)
     lerr = float(np.abs(lg - lse_o).max())
-    assert err <= TOL_OUT[dtype], (err, float(np.abs(og - out_o).max()))
+    print(f"[{dtype}] max|dO| {raw:.3e}  vs bf16(O_ref) {vs_rounded:.3e}  beyond the output's rounding "
+          f"{beyond_rounding:.3e}  scaled {err:.3e}  max|dLSE| {lerr:.3e}")
+    assert beyond_rounding <= TOL_OUT[dtype], (beyond_rounding, raw, vs_rounded)
+    assert err <= TOL_OUT[dtype], (err, raw)
     assert lerr <= TOL_LSE, lerr
     return err, lerr
 

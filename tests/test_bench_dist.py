@@ -49,7 +49,8 @@ def test_two_gloo_ranks_reduce_max_and_sum():
 
 def test_reference_arm_runs_on_rank0_only_and_prints_one_line():
     env = dict(os.environ, RANK="1", WORLD_SIZE="2")
-    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--workload", "tiny",
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--impl", "reference",
+                        "--workload", "tiny",
                         "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"], env=env, capture_output=True,
                        text=True, timeout=300)
     assert r.returncode == 0 and r.stdout.strip() == ""
@@ -67,3 +68,23 @@ def test_reference_arm_runs_on_rank0_only_and_prints_one_line():
         assert k in d, k
     assert d["impl"] == "reference" and d["cpu_baseline"]["kind"] == "oracle"
     assert d["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_gpus_flag_against_the_launcher():
+    """--gpus N must agree with the launcher's WORLD_SIZE; without a launcher,
+    --gpus 2 starts two ranks itself (here on the reference arm, which rank 0
+    alone runs), so exactly one JSON line comes out."""
+    args = ["--impl", "reference", "--workload", "tiny", "--steps", "1", "--warmup", "0", "--cpu-seconds", "1"]
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", *args], env=env,
+                       capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE" in r.stderr
+    env = {k: v for k, v in os.environ.items() if k not in ("RANK", "WORLD_SIZE", "LOCAL_RANK", "MASTER_ADDR",
+                                                             "MASTER_PORT")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", *args], env=env,
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    import json
+    lines = [x for x in r.stdout.splitlines() if x.strip().startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["impl"] == "reference"

@@ -77,8 +77,9 @@ def test_paged_equals_packed(name):
     assert torch.equal(lse.view(torch.int32), lse_ref.view(torch.int32))
 
 
-def test_paged_attention_matches_oracle_through_the_gather():
-    w, ps = CASES["varlen_page64"]
+@pytest.mark.parametrize("name", ["varlen_page64", "fp8_page256"])
+def test_paged_attention_matches_oracle_through_the_gather(name):
+    w, ps = CASES[name]
     cu = w.cu_seqlens()
     inp = I.make_inputs(w, device="cuda")
     qkv = make_gpu_qkv(b, inp, cu)
@@ -86,10 +87,25 @@ def test_paged_attention_matches_oracle_through_the_gather():
     _, _, rp, ci, _ = b.stem_prefill(qkv, params)
     kp, table = to_pages(inp["k"], cu, ps, np.random.default_rng(3))
     vp, _ = to_pages(inp["v"], cu, ps, np.random.default_rng(3))
-    out, lse, _ = b.stem_bsa_fwd_paged(qkv, b.paged_kv(kp.cuda(), vp.cuda(), table.cuda(), ps), params, rp, ci)
-    q = O.dequant(I.raw_bits(inp["q"].cpu()), "bf16")
-    kg = O.gather_paged(O.dequant(I.raw_bits(kp), "bf16"), table.numpy(), cu, ps)
-    vg = O.gather_paged(O.dequant(I.raw_bits(vp), "bf16"), table.numpy(), cu, ps)
+    out, lse, ws = b.stem_bsa_fwd_paged(qkv, b.paged_kv(kp.cuda(), vp.cuda(), table.cuda(), ps), params, rp, ci)
+    torch.cuda.synchronize()
+    assert b.stem_read_device_status(ws) == 0
+
+    def pool_f64(pool, name):
+        """fp64 values of a [P, page_size, H, d] pool (fp8: times the per-head scale)."""
+        flat = pool.reshape(-1, *pool.shape[2:])
+        if w.dtype == "bf16":
+            x = O.dequant(I.raw_bits(flat), "bf16")
+        else:
+            x = O.dequant(I.raw_bits(flat), "fp8", inp[name + "_scale"].cpu().numpy())
+        return x.reshape(pool.shape)
+
+    if w.dtype == "bf16":
+        q = O.dequant(I.raw_bits(inp["q"].cpu()), "bf16")
+    else:
+        q = O.dequant(I.raw_bits(inp["q"].cpu()), "fp8", inp["q_scale"].cpu().numpy())
+    kg = O.gather_paged(pool_f64(kp, "k"), table.numpy(), cu, ps)
+    vg = O.gather_paged(pool_f64(vp, "v"), table.numpy(), cu, ps)
     ro, rl = O.bsa(q, kg, vg, cu, rp.cpu().numpy(), ci.cpu().numpy(), O.Params(**w.params()))
     check_attention(out, lse, ro, rl, w.dtype)
 

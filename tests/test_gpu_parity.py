@@ -130,6 +130,50 @@ def test_select_ties_go_to_lowest_index():
     assert np.array_equal(gci.cpu().numpy(), oci)
 
 
+def test_select_signed_zeros_tie_by_index():
+    """Caller-given scores whose selection threshold falls on a -0.0 at a lower
+    key block and a +0.0 at a higher one: the two are equal numbers, so the
+    lower index is taken (the oracle's rule), not the +0.0."""
+    c = get_case("multi_tile")
+    rng = np.random.default_rng(5)
+    s32 = c.ref_scores.astype(np.float32)
+    bud = O.budgets(c.cu, c.p)
+    seqs, nbtot = O.seq_blocks(c.cu)
+    planted = []
+    for h in range(c.w.num_q_heads):
+        for (_, _, nb, g0) in seqs:
+            for i in range(nb):
+                F = set(O.forced_blocks(i, c.p.sink_blocks, c.p.window_blocks))
+                cand = [j for j in range(i + 1) if j not in F]
+                m = min(max(int(bud[g0 + i]) - len(F), 0), len(cand))
+                if m < 1 or len(cand) < m + 1:
+                    continue
+                perm = rng.permutation(cand)
+                top, zeros, rest = perm[:m - 1], sorted(perm[m - 1:m + 1]), perm[m + 1:]
+                row = s32[h, g0 + i]
+                row[top] = 1.0 + rng.random(len(top)).astype(np.float32)
+                row[zeros[0]] = np.float32(-0.0)
+                row[zeros[1]] = np.float32(0.0)
+                row[rest] = -1.0 - rng.random(len(rest)).astype(np.float32)
+                planted.append((h * nbtot + g0 + i, zeros[0], zeros[1]))
+    assert len(planted) > 20
+    gb, grp, gci, ws = b.stem_select(c.qkv, c.params, torch.from_numpy(s32).cuda())
+    assert b.stem_read_device_status(ws) == 0
+    ob, orp, oci = O.select(s32.astype(np.float64), c.cu, c.p, hkv=c.w.num_kv_heads)
+    for (r, lo, hi) in planted:
+        row = oci[orp[r]:orp[r + 1]].tolist()
+        assert lo in row and hi not in row
+    assert np.array_equal(grp.cpu().numpy(), orp)
+    assert np.array_equal(gci.cpu().numpy(), oci)
+    # the same rows through the KV-group-shared selection (max over the group)
+    params1 = b.make_params(**dict(c.w.params(), list_mode=1))
+    _, grp1, gci1, _ = b.stem_select(c.qkv, params1, torch.from_numpy(s32).cuda())
+    p1 = O.Params(**dict(c.w.params(), list_mode=1))
+    _, orp1, oci1 = O.select(s32.astype(np.float64), c.cu, p1, hkv=c.w.num_kv_heads)
+    assert np.array_equal(grp1.cpu().numpy(), orp1)
+    assert np.array_equal(gci1.cpu().numpy(), oci1)
+
+
 @pytest.mark.parametrize("name", list(CASES))
 def test_prefill_end_to_end(name):
     c = get_case(name)

@@ -178,6 +178,13 @@ def test_selection_ties_nan_and_structure():
             sel = ci[rp[r]:rp[r + 1]].tolist()
             assert len(sel) == bud[r] and sel == sorted(set(sel))
             assert set(O.forced_blocks(i, 2, 3)) <= set(sel) and max(sel) == i
+    # -0.0 and +0.0 are equal numbers: between them the lower index wins,
+    # whichever of the two carries the sign bit
+    z = np.array([-1.0, 0.0, -0.0, 2.0, -0.0, 0.0, -3.0, 7.0])
+    assert O.select_row(z, 7, 3, 0, 1) == [1, 3, 7]
+    z2 = np.array([-1.0, -0.0, 0.0, 2.0, 0.0, -0.0, -3.0, 7.0])
+    assert O.select_row(z2, 7, 3, 0, 1) == [1, 3, 7]
+    assert O.select_row(z2, 7, 4, 0, 1) == [1, 2, 3, 7]
     # rho = 1, mu = 1 selects every causal block
     bud, rp, ci = O.select(sc, cu, O.Params(keep_ratio=1.0, mu=1.0, sink_blocks=0, window_blocks=1))
     rp2, ci2 = O.full_csr(cu, 3)

@@ -37,12 +37,27 @@ def test_noalloc_matches_workspace_prefill_on_two_calls(dtype):
         out, lse, rp, ci = b.stem_prefill_noalloc(qkv, params)
         torch.cuda.synchronize()
         assert b.stem_read_device_status(ws) == 0
+        assert b.stem_noalloc_read_device_status() == 0  # the built-in workspace's own status word
         assert torch.equal(rp, ref_rp) and torch.equal(ci, ref_ci)
         err = out_error(out.float().cpu().numpy(), ref_out.float().cpu().numpy())
         assert err <= TOL_OUT[dtype]
         assert float((lse - ref_lse).abs().max()) <= TOL_LSE
         # same kernels on the same inputs: the results are in fact identical
         assert torch.equal(out, ref_out) and torch.equal(lse, ref_lse)
+
+
+def test_noalloc_status_word_reads_ok_on_any_stream_of_the_device():
+    """The built-in workspace's status word (where a timed-out wait or a
+    malformed list entry would be recorded; a valid prefill produces neither)
+    reads STEM_OK after calls on the default stream and on a side stream of
+    the same device, which the device check accepts."""
+    w, qkv, params = _case(303)
+    b.stem_prefill_noalloc(qkv, params)
+    assert b.stem_noalloc_read_device_status() == 0
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        b.stem_prefill_noalloc(qkv, params, stream=s)
+    assert b.stem_noalloc_read_device_status(s) == 0
 
 
 def test_noalloc_rejects_problems_larger_than_its_workspace():
