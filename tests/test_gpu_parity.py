@@ -247,7 +247,8 @@ def test_results_are_deterministic():
 @pytest.mark.parametrize("name", ["group_lists", "group_lists_odd_group", "group_lists_fp8"])
 def test_shared_list_pairs_equal_the_one_row_kernel(name):
     """With shared lists the attention runs two query heads per CTA on one
-    staged K/V stream; per row it is the same arithmetic as one row per CTA."""
+    staged K/V stream; per row it is the same arithmetic as one row per CTA,
+    so the results are bit-identical (and match the oracle)."""
     c = get_case(name)
     _, _, rp, ci, _ = b.stem_prefill(c.qkv, c.params)
     out_pair, lse_pair, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, ci)
@@ -257,6 +258,8 @@ def test_shared_list_pairs_equal_the_one_row_kernel(name):
     assert b.stem_read_device_status(ws2) == 0
     assert torch.equal(out_pair.view(torch.int16), out_row.view(torch.int16))
     assert torch.equal(lse_pair.view(torch.int32), lse_row.view(torch.int32))
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp.cpu().numpy(), ci.cpu().numpy(), c.p)
+    check_attention(out_pair, lse_pair, ro, rl, c.w.dtype)
 
 
 def test_shared_list_mode_reports_rows_that_differ():
