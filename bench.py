@@ -57,11 +57,15 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-fp8", action="store_true", help="skip the e4m3 attention timing of the default mode")
     ap.add_argument("--cpu-seconds", type=float, default=15.0, help="bounded oracle sample, seconds")
-    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality", "variants"], default="default",
+    ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality", "variants", "once"], default="default",
                     help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack; "
                          "quality: reconstruction error against dense attention (32K); "
-                         "variants: the 128K step with the standardized bonus and KV-group-shared lists")
+                         "variants: the 128K step with the standardized bonus and KV-group-shared lists; "
+                         "once: one untimed step of --workload (the command profilers wrap)")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
+    ap.add_argument("--separate-select", action="store_true",
+                    help="mode once: stem_score then stem_select (the selection kernel of its own) instead of the "
+                         "fused stem_score_select")
     return ap.parse_args(argv)
 
 
@@ -877,6 +881,29 @@ def launch_ranks(args, argv) -> int | None:
     return subprocess.run(cmd).returncode
 
 
+def run_once(args):
+    """One step of the workload (stem_score_select, then stem_bsa_fwd) and
+    nothing else: the smallest program that launches each of the step's
+    kernels once, for profilers.  Prints the device status."""
+    import torch
+    from block_sparse_attention_stem_b200 import binding as b
+    from block_sparse_attention_stem_b200 import inputs as I
+    w = bench_workload(I, args)
+    inp = I.make_inputs(w, device="cuda")
+    qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w.cu_seqlens(), q_scale=inp["q_scale"], k_scale=inp["k_scale"],
+                     v_scale=inp["v_scale"], cu_seqlens_dev=inp["cu_seqlens"])
+    params = b.make_params(**w.params())
+    if args.separate_select:
+        scores, _, ws = b.stem_score(qkv, params)
+        budgets, row_ptr, col_idx, _ = b.stem_select(qkv, params, scores, ws=ws)
+    else:
+        scores, budgets, row_ptr, col_idx, ws = b.stem_score_select(qkv, params)
+    out, lse, _ = b.stem_bsa_fwd(qkv, params, row_ptr, col_idx, ws=ws)
+    torch.cuda.synchronize()
+    print(json.dumps({"mode": "once", "workload": w.name, "dtype": w.dtype,
+                      "status": b.stem_status_string(b.stem_read_device_status(ws))}), flush=True)
+
+
 def main(argv=None):
     args = parse_args(argv)
     rc = launch_ranks(args, argv)
@@ -892,6 +919,8 @@ def main(argv=None):
         run_variants(args)
     elif args.mode == "fp8stack":
         run_fp8stack(args)
+    elif args.mode == "once":
+        run_once(args)
     else:
         run_ours(args)
 

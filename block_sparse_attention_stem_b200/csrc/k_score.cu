@@ -300,8 +300,8 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
       //    block, scale, bonus (lane k holds the tile's k-th key block's), store
       const int jl = J * kbt + lane;
       const float bl = (lane < kbt && jl < nb) ? bonus[jl] : 0.f;
-#pragma unroll 1
-      for (int k = 0; k < kbh; ++k) {
+#pragma unroll
+      for (int k = 0; k < kbh; ++k) {  // unrolled, so that pooled[] stays in registers
         float v = row_valid ? pooled[k] : ninf;
 #pragma unroll
         for (int off = gpb / 2; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
