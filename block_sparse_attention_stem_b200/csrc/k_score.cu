@@ -341,7 +341,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
         if (ib >= nb) break;
         const size_t r = static_cast<size_t>(h) * args.nbtot + batch.g0[seq] + ib;
         warp_select_row(args.scores + r * static_cast<size_t>(args.nb_max), ib, args.budgets[r], args.sink,
-                        args.window, keys, hist, args.col_idx + args.row_ptr[r]);
+                        args.window, keys, hist, args.col_idx, args.row_ptr, r);
       }
     }
   }

@@ -5,9 +5,9 @@
 // HPC-BSA article §3.1 (the compacted, ascending list the attention walks):
 // keep the forced blocks F, then the m = min(max(b - |F|, 0), c - |F|) best
 // other causal blocks by (score descending, index ascending), NaN ranked as
-// -inf; write them in ascending order.  The same rule as select_kernel, at
-// warp granularity, so the scoring kernel can select the rows it has just
-// scored.
+// -inf; write them in ascending order.  One warp per row: the scoring kernel
+// selects the rows it has just scored with it, and select_kernel runs it on
+// given scores.
 #pragma once
 
 #include "stem_device.cuh"
@@ -37,10 +37,17 @@ __device__ __forceinline__ int warp_exclusive_scan(int x) {
 }
 
 // row: the row's block scores (index = key block, local to the sequence), at
-// least i + 1 of them; keys: this warp's scratch (>= i + 1 entries); hist: this
-// warp's scratch of 256 ints; out: where the list starts (b entries).
-static __device__ __noinline__ void warp_select_row(const float* __restrict__ row, int i, int b, int sink, int window,
-                                             uint32_t* keys, int* hist, int32_t* __restrict__ out) {
+// least i + 1 of them; with group > 1 the rows of the group's other query
+// heads follow at multiples of head_stride, and a block's key is the best of
+// the group's scores (order_key is monotone and maps NaN below every number).
+// keys: this warp's scratch (>= i + 1 entries); hist: this warp's scratch of
+// 256 ints; the list (b entries, ascending) is written to
+// col_idx + row_ptr[r + e row_stride] for each of the group's heads e.
+static __device__ __noinline__ void warp_select_row_group(const float* __restrict__ row, size_t head_stride,
+                                                          int group, int i, int b, int sink, int window,
+                                                          uint32_t* keys, int* hist, int32_t* __restrict__ col_idx,
+                                                          const int32_t* __restrict__ row_ptr, size_t r,
+                                                          size_t row_stride) {
   const int lane = lane_id();
   const int c = i + 1;
   const int nforced = static_cast<int>(forced_count(i, sink, window));
@@ -50,7 +57,11 @@ static __device__ __noinline__ void warp_select_row(const float* __restrict__ ro
   uint32_t thr = 0u;
   int take_eq = 0;  // candidates equal to thr to take, lowest index first
   if (m > 0 && !all) {
-    for (int j = lane; j < c; j += 32) keys[j] = order_key(row[j]);
+    for (int j = lane; j < c; j += 32) {
+      uint32_t k = order_key(row[j]);
+      for (int e = 1; e < group; ++e) k = max(k, order_key(row[e * head_stride + j]));
+      keys[j] = k;
+    }
     __syncwarp();
     // radix select of the m-th largest candidate key, 8 bits per pass
     uint32_t prefix = 0u;
@@ -119,13 +130,22 @@ static __device__ __noinline__ void warp_select_row(const float* __restrict__ ro
     int e = eq_before;
     for (int j = j0; j < j1; ++j) n_sel += take(j, e);
   }
-  int pos = warp_exclusive_scan(n_sel);
-  {
-    int e = eq_before;
+  const int pos0 = warp_exclusive_scan(n_sel);
+  for (int h = 0; h < group; ++h) {
+    int32_t* __restrict__ out = col_idx + row_ptr[r + h * row_stride];
+    int e = eq_before, pos = pos0;
     for (int j = j0; j < j1; ++j)
       if (take(j, e)) out[pos++] = j;
   }
   __syncwarp();
+}
+
+// One query head's row (the fused selection of the scoring kernel).
+static __device__ __forceinline__ void warp_select_row(const float* __restrict__ row, int i, int b, int sink,
+                                                       int window, uint32_t* keys, int* hist,
+                                                       int32_t* __restrict__ col_idx,
+                                                       const int32_t* __restrict__ row_ptr, size_t r) {
+  warp_select_row_group(row, 0, 1, i, b, sink, window, keys, hist, col_idx, row_ptr, r, 0);
 }
 
 }  // namespace stem
