@@ -277,3 +277,31 @@ def test_shared_list_mode_reports_rows_that_differ():
     ci_h[rp_h[r]:rp_h[r + 1]] = np.sort(row)
     out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, torch.from_numpy(ci_h).cuda())
     assert b.stem_read_device_status(ws) == 7  # STEM_ERR_BAD_BLOCKLIST
+
+
+@pytest.mark.parametrize("list_mode", [0, 1])
+def test_select_long_rows_on_given_scores(list_mode):
+    """The standalone selection on rows of up to 2,500 key blocks (each warp's
+    keys and histogram need more than the default 48 KB of shared memory per
+    CTA), per query head and with KV-group-shared lists: seeded fp32 scores
+    with repeated values (ties) and a few NaN, selected by the GPU and by the
+    oracle on the very same values; the lists must be identical."""
+    nb = 2500
+    w = I.Workload(name="long_select", seqlens=[nb * 128 - 77], num_q_heads=4, num_kv_heads=2, seed=61,
+                   keep_ratio=0.3, mu=0.7, beta=0.2, sink_blocks=2, window_blocks=3, list_mode=list_mode)
+    cu = w.cu_seqlens()
+    q = torch.zeros(1, w.num_q_heads, 128, dtype=torch.bfloat16, device="cuda")  # scores are given: never read
+    qkv = b.make_qkv(q, q[:, :w.num_kv_heads].contiguous(), q[:, :w.num_kv_heads].contiguous(), cu,
+                     cu_seqlens_dev=torch.tensor(cu, dtype=torch.int32, device="cuda"))
+    qkv.desc.total_tokens = cu[-1]
+    params = b.make_params(**w.params())
+    rng = np.random.default_rng(7)
+    s32 = (np.round(rng.standard_normal((w.num_q_heads, nb, nb)) * 8) / 8).astype(np.float32)
+    s32[rng.random(s32.shape) < 0.001] = np.nan
+    gb, grp, gci, ws = b.stem_select(qkv, params, torch.from_numpy(s32).cuda())
+    torch.cuda.synchronize()
+    assert b.stem_read_device_status(ws) == 0
+    ob, orp, oci = O.select(s32.astype(np.float64), cu, O.Params(**w.params()), hkv=w.num_kv_heads)
+    assert np.array_equal(gb.cpu().numpy(), ob)
+    assert np.array_equal(grp.cpu().numpy(), orp)
+    assert np.array_equal(gci.cpu().numpy(), oci)
