@@ -4,10 +4,16 @@
 // beta * max(0, log ||V_j||^2); the value norms are max-pooled per key block.
 //   vbonus[hk][g0 + j] = beta * max(0, ln max_{t in block j} ||v_t||^2)
 //
-// One CTA per key block reads the block's 128 tokens x Hkv heads x 128 values
-// (256 KB bf16, contiguous in the packed [T, Hkv, d] layout) once with 16-byte
+// Two CTAs per key block, each taking half of the KV heads, read the block's
+// 128 tokens x Hkv heads x 128 values (256 KB bf16 in the packed [T, Hkv, d]
+// layout; each CTA reads 1 KB of every 2 KB token row) once with 16-byte
 // loads; 16 (bf16) or 8 (fp8) lanes cover one (token, head) row of 128
-// values, and each thread keeps four rows' loads in flight.  The arithmetic
+// values, and each thread keeps eight rows' loads in flight.  Measured at
+// 8 KV heads (one launch each, cold L2): with four rows in flight and one CTA
+// per block the pass took 65.5 us at 131072 tokens; eight rows 58.6 us, and
+// two head groups 57.2 us there and 18.9 us instead of 25.7 us at 32768
+// tokens, where one CTA per block leaves the SMs too few loads in flight
+// (four head groups: 56.9 / 20.4 us; eight: 60.5 / 20.8 us).  The arithmetic
 // per byte is small but not free (widening, packed FMAs, the row's lane
 // reduction), so it is kept to a few instructions per 16-byte load.
 #include <cuda_bf16.h>
@@ -20,10 +26,13 @@ namespace stem {
 
 template <bool kFp8>
 __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const uint8_t* __restrict__ v,
-                                                    const float* __restrict__ v_scale, int hkv, int hk0, int nhk,
-                                                    int nbtot, float beta, bool raw_log,
-                                                    float* __restrict__ vbonus) {
+                                                    const float* __restrict__ v_scale, int hkv, int hk_first,
+                                                    int nhk_all, int heads_per_cta, int nbtot, float beta,
+                                                    bool raw_log, float* __restrict__ vbonus) {
   extern __shared__ unsigned int s_max[];  // [nhk] bit patterns of non-negative floats (KV heads hk0 ..)
+  // this CTA's KV heads: hk0 .. hk0 + nhk - 1 (group blockIdx.y of the launch's range)
+  const int hk0 = hk_first + static_cast<int>(blockIdx.y) * heads_per_cta;
+  const int nhk = min(heads_per_cta, hk_first + nhk_all - hk0);
   const int s = find_seq(batch, blockIdx.x);
   const int j = blockIdx.x - batch.item0[s];
   const int t0 = j * kBlock;
@@ -37,11 +46,11 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
   const int sub = threadIdx.x % kLanesPerRow;
   const int row_step = blockDim.x / kLanesPerRow;
   const uint8_t* base = v + (static_cast<size_t>(batch.tok0[s]) + t0) * hkv * kHeadDim * kElt;
-  // four rows per thread in flight: their loads are issued before any of them
+  // eight rows per thread in flight: their loads are issued before any of them
   // is reduced (the trip count is uniform across a warp, so every lane takes
   // part in the shuffles).  Row r is (token r / nhk, head r % nhk); the pair
   // is advanced by row_step without a division per row.
-  constexpr int kUnroll = 4;
+  constexpr int kUnroll = 8;
   const int first = threadIdx.x / kLanesPerRow;
   const int q_step = row_step / nhk, r_step = row_step % nhk;
   int quo = first / nhk, rem = first % nhk;
@@ -111,13 +120,15 @@ cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_sc
                          int nhk, int nbtot, float beta, bool raw_log, float* vbonus, cudaStream_t stream) {
   const int items = batch.item0[batch.n];
   if (items == 0 || nhk <= 0) return cudaSuccess;
-  const size_t smem = sizeof(unsigned int) * static_cast<size_t>(nhk);
+  const int heads_per_cta = (nhk + 1) / 2;  // two head groups (one when nhk = 1)
+  const dim3 grid(items, (nhk + heads_per_cta - 1) / heads_per_cta);
+  const size_t smem = sizeof(unsigned int) * static_cast<size_t>(heads_per_cta);
   if (fp8)
-    vnorm_kernel<true><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                     nbtot, beta, raw_log, vbonus);
+    vnorm_kernel<true><<<grid, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
+                                                    heads_per_cta, nbtot, beta, raw_log, vbonus);
   else
-    vnorm_kernel<false><<<items, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                      nbtot, beta, raw_log, vbonus);
+    vnorm_kernel<false><<<grid, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
+                                                     heads_per_cta, nbtot, beta, raw_log, vbonus);
   return cudaGetLastError();
 }
 
