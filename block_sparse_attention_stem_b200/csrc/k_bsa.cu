@@ -79,9 +79,75 @@ struct BsaSmem {
   int abort;
 };
 
+// 64-token blocks: the lists of query blocks 2p and 2p + 1 (rows 0-63 and
+// 64-127 of the CTA's 128-token tile) as two bitmaps of key blocks in the
+// list storage (words 0 .. 1023 and 1024 .. 2047); *nunits = size of their
+// union.  Valid entries as for the staged list (0 <= j <= the row's block,
+// above the previous valid entry); a malformed list is compacted entry by
+// entry and reported.  One whole warp.
+constexpr int kBitmapWords = kMaxBitmapBlocks / 32;
+static_assert(2 * kBitmapWords <= kMaxList, "two bitmaps must fit the list storage");
+
+__device__ void stage_bitmaps(const int32_t* __restrict__ col, int beg0, int end0, int i0, int beg1, int end1,
+                              int i1, int nwords, uint32_t* bm, int* nunits, int* status) {
+  const int lane = lane_id();
+  for (int w = lane; w < nwords; w += 32) {
+    bm[w] = 0u;
+    bm[kBitmapWords + w] = 0u;
+  }
+  __syncwarp();
+  for (int e = 0; e < 2; ++e) {
+    const int beg = e ? beg1 : beg0, end = e ? end1 : end0, i = e ? i1 : i0;
+    uint32_t* b = bm + e * kBitmapWords;
+    bool good = true;
+    for (int p0 = beg; p0 < end; p0 += 32) {
+      const int p = p0 + lane;
+      const int j = p < end ? __ldg(col + p) : 0;
+      int before = __shfl_up_sync(0xffffffffu, j, 1);
+      if (lane == 0) before = p0 > beg ? __ldg(col + p0 - 1) : -1;
+      if (__any_sync(0xffffffffu, p < end && (j < 0 || j > i || j <= before))) {
+        good = false;
+        break;
+      }
+      if (p < end) atomicOr(b + (j >> 5), 1u << (j & 31));
+    }
+    __syncwarp();
+    if (!good && lane == 0) {
+      set_status(status, STEM_ERR_BAD_BLOCKLIST_CODE);
+      for (int w = 0; w < nwords; ++w) b[w] = 0u;
+      int prev = -1, j = 0;
+      for (int p = next_valid(col, beg, end, prev, i, &j); p < end; p = next_valid(col, p + 1, end, prev, i, &j)) {
+        b[j >> 5] |= 1u << (j & 31);
+        prev = j;
+      }
+    }
+    __syncwarp();
+  }
+  int n = 0;
+  for (int w = lane; w < nwords; w += 32) n += __popc(bm[w] | bm[kBitmapWords + w]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) n += __shfl_xor_sync(0xffffffffu, n, off);
+  if (lane == 0) *nunits = n;
+}
+
+// Walks the union of the two bitmaps in ascending key-block order.
+struct BitmapCursor {
+  int w = -1;
+  uint32_t bits = 0u;
+  __device__ __forceinline__ int next(const uint32_t* bm) {
+    while (bits == 0u && w + 1 < kBitmapWords) {
+      ++w;
+      bits = bm[w] | bm[kBitmapWords + w];
+    }
+    const int b = __ffs(bits) - 1;
+    bits &= bits - 1u;
+    return w * 32 + b;
+  }
+};
+
 }  // namespace
 
-template <bool kFp8>
+template <bool kFp8, bool kB64>
 __global__ void __launch_bounds__(kBsaThreads, 2)
     bsa_kernel(const __grid_constant__ BsaMaps maps, const SeqBatch batch, const BsaArgs args) {
   using Cfg = BsaCfg<kFp8>;
@@ -96,21 +162,38 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
   const int G = args.hq / args.hkv;
   // Rows of a sequence in KV-head-major order: KV head, then query blocks
   // descending (longest rows first), then the query heads of the group.
+  // tl.i: the 128-token query tile (query block i, or with 64-token blocks
+  // query blocks 2i and 2i + 1, whose second CSR range is beg1 .. end1)
+  const int ntiles = kB64 ? (nb + 1) / 2 : nb;
   Tile tl;
+  int beg1 = 0, end1 = 0;
   {
     const int it = blockIdx.x - batch.item0[seq];
-    const int hk_of = args.hk0 + it / (G * nb);
-    const int rem = it % (G * nb);
+    const int hk_of = args.hk0 + it / (G * ntiles);
+    const int rem = it % (G * ntiles);
     tl.valid = true;
-    tl.i = nb - 1 - rem / G;
+    tl.i = ntiles - 1 - rem / G;
     tl.h = hk_of * G + rem % G;
     tl.hk = tl.h / G;
-    const size_t r = static_cast<size_t>(tl.h) * args.nbtot + batch.g0[seq] + tl.i;
+    const size_t r = static_cast<size_t>(tl.h) * args.nbtot + batch.g0[seq] + (kB64 ? 2 * tl.i : tl.i);
     tl.beg = args.row_ptr[r];
     tl.end = args.row_ptr[r + 1];
+    if (kB64 && 2 * tl.i + 1 < nb) {
+      beg1 = args.row_ptr[r + 1];
+      end1 = args.row_ptr[r + 2];
+    }
   }
+  uint32_t* bitmaps = reinterpret_cast<uint32_t*>(sm.list);
 
-  if (warp == kKProducerWarp) stage_list(args.col_idx, tl, sm.list, &sm.nvalid, &sm.in_smem, args.status);
+  if (warp == kKProducerWarp) {
+    if constexpr (kB64) {
+      stage_bitmaps(args.col_idx, tl.beg, tl.end, 2 * tl.i, beg1, end1, 2 * tl.i + 1, (nb + 31) / 32, bitmaps,
+                    &sm.nvalid, args.status);
+      if (lane_id() == 0) sm.in_smem = 1;
+    } else {
+      stage_list(args.col_idx, tl, sm.list, &sm.nvalid, &sm.in_smem, args.status);
+    }
+  }
   if (threadIdx.x == 0) {
     mbar_init(&sm.q_full, 1);
     for (int b = 0; b < 2; ++b) {
@@ -154,21 +237,23 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
         for (int hh = 0; hh < Cfg::kKSlabs; ++hh)
           tma_load_3d(sm.q + hh * 16384, &maps.q[seq], &sm.q_full, hh * 64, tl.h, tl.i * kBlock);
       }
-      const int H = 2 * N;
+      const int H = kB64 ? N : 2 * N;  // 64-key units
       ListCursor cur(tl.beg);
+      BitmapCursor bcur;
       int j = 0, issued = 0;
       for (int h = 0; h < H; ++h) {
         if (h >= 2) {
           uint64_t* freed = is_v ? &sm.v_free[h & 1] : &sm.s_full[h & 1];
           if (!mbar_wait(freed, ((h - 2) >> 1) & 1, abort, args.status)) break;
         }
-        if ((h & 1) == 0) j = cur.next(sm.list, list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
+        if (kB64) j = bcur.next(bitmaps);
+        else if ((h & 1) == 0) j = cur.next(sm.list, list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
         uint8_t* dst = is_v ? sm.v[h & 1] : sm.k[h & 1];
         uint64_t* bar = is_v ? &sm.v_full[h & 1] : &sm.k_full[h & 1];
-        // token row of the half: in the sequence, or through the page table (a
-        // 64-key half never straddles a page; a page number outside the pool
+        // token row of the unit: in the sequence, or through the page table (a
+        // 64-key unit never straddles a page; a page number outside the pool
         // reads zeros)
-        int row = j * kBlock + (h & 1) * kHalf;
+        int row = kB64 ? j * kHalf : j * kBlock + (h & 1) * kHalf;
         if (paged) row = __ldg(pages + row / args.page_size) * args.page_size + row % args.page_size;
         mbar_arrive_expect_tx(bar, half_bytes);
         for (int hh = 0; hh < slabs; ++hh) tma_load_3d(dst + hh * (kHalf * 128), m, bar, hh * 64, tl.hk, row);
@@ -191,7 +276,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
       const uint32_t idesc_o = make_idesc(kFp8 ? 0u : 1u, 1u, 128u, 128u);  // kind::f16: f16 (0) or bf16 (1)
       const uint32_t sq = smem_u32(sm.q);
       const uint32_t o_tmem = tmem + 128;
-      const int H = 2 * N;
+      const int H = kB64 ? N : 2 * N;
       auto issue_s = [&](int h) -> bool {  // S_h = Q K_h^T into buffer h % 2
         if (!mbar_wait(&sm.k_full[h & 1], (h >> 1) & 1, abort, args.status)) return false;
         tc_fence_after();
@@ -228,7 +313,8 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
       };
       // S_0, S_1, then per half h: P_h V_h and S_{h+2} (into the buffer P_h
       // V_h just read: the tensor core runs one issuer's products in order)
-      bool ok = mbar_wait(&sm.q_full, 0, abort, args.status) && issue_s(0) && issue_s(1);
+      // (with 64-token blocks a tile may have a single unit)
+      bool ok = mbar_wait(&sm.q_full, 0, abort, args.status) && issue_s(0) && (H < 2 || issue_s(1));
       for (int h = 0; h < H && ok; ++h) {
         ok = issue_pv(h);
         if (ok && h + 2 < H) ok = issue_s(h + 2);
@@ -255,19 +341,46 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
     float l = 0.f;       // row sum of exp2(s c - m_ref)
     bool ok = true;
     ListCursor cur(tl.beg);
-    for (int n = 0; n < N && ok; ++n) {
-      const int j = cur.next(sm.list, list_in_smem, n, args.col_idx, tl.end, tl.i);
-      const bool diag = (j == tl.i);
+    BitmapCursor bcur;
+    const int H = kB64 ? N : 2 * N;  // 64-key units
+    int j = 0;
 #pragma unroll 1
-      for (int half = 0; half < 2; ++half) {
-        const int h = 2 * n + half;
+    for (int h = 0; h < H && ok; ++h) {
+      {
+        const int half = h & 1;  // S buffer of the unit
+        // koff: the unit's first key minus the tile's first token (>= 0 only
+        // on the diagonal, where keys above a row's token are masked)
+        int koff;
+        bool member = true;  // the unit is in the list of this warp's rows
+        if constexpr (kB64) {
+          j = bcur.next(bitmaps);
+          koff = j * kHalf - tl.i * kBlock;
+          member = ((bitmaps[(q4 >> 1) * kBitmapWords + (j >> 5)] >> (j & 31)) & 1u) != 0u;
+        } else {
+          if (half == 0) j = cur.next(sm.list, list_in_smem, h >> 1, args.col_idx, tl.end, tl.i);
+          koff = (j == tl.i) ? half * kHalf : -kBlock;
+        }
+        const bool diag = koff >= 0;
         const uint32_t s_tmem = s_base + kHalf * half;
-        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[half], n & 1, abort, args.status))) {
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.s_full[half], (h >> 1) & 1, abort, args.status))) {
           ok = false;
           break;
         }
         tc_fence_after();
-        // the half's 64 scores, loaded once and kept in registers
+        if (kB64 && !member) {
+          // the other query block's unit: P = 0 for these rows
+          uint32_t z[16];
+#pragma unroll
+          for (int x = 0; x < 16; ++x) z[x] = 0u;
+          tmem_st16(s_tmem, z);
+          tmem_st16(s_tmem + 16, z);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.p_full[half]);
+          continue;
+        }
+        // the unit's 64 scores, loaded once and kept in registers
         uint32_t rr[2][32];
         tmem_ld32(s_tmem, rr[0]);
         tmem_ld32(s_tmem + 32, rr[1]);
@@ -277,7 +390,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
           for (int ch = 0; ch < 2; ++ch)
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              if (half * kHalf + ch * 32 + x > row) rr[ch][x] = 0xff800000u;  // -inf -> p = 0
+              if (koff + ch * 32 + x > row) rr[ch][x] = 0xff800000u;  // -inf -> p = 0
         }
         float m4[4];
 #pragma unroll
@@ -300,7 +413,7 @@ __global__ void __launch_bounds__(kBsaThreads, 2)
           const float alpha = (m_ref == ninf) ? 0.f : fast_exp2(m_ref - m_new);
           l *= alpha;
           if (h >= 1) {
-            // O holds P V up to half h-1: let that product finish first
+            // O holds P V up to unit h-1: let that product finish first
             if (!__all_sync(0xffffffffu,
                             mbar_wait(&sm.v_free[(h - 1) & 1], ((h - 1) >> 1) & 1, abort, args.status))) {
               ok = false;
@@ -390,23 +503,27 @@ size_t bsa_smem_bytes(bool fp8) {
   return need > (size_t(80) << 10) ? need : (size_t(80) << 10);
 }
 
+template <bool kFp8, bool kB64>
+static cudaError_t launch_bsa_t(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, int items,
+                                cudaStream_t stream) {
+  const size_t smem = bsa_smem_bytes(kFp8);
+  const cudaError_t e = cudaFuncSetAttribute(bsa_kernel<kFp8, kB64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  bsa_kernel<kFp8, kB64><<<items, kBsaThreads, smem, stream>>>(maps, batch, args);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_bsa(const BsaMaps& maps, const SeqBatch& batch, const BsaArgs& args, bool fp8,
                        cudaStream_t stream) {
   const int items = batch.item0[batch.n];
   if (items == 0) return cudaSuccess;
-  const size_t smem = bsa_smem_bytes(fp8);
-  cudaError_t e;
-  if (fp8) {
-    e = cudaFuncSetAttribute(bsa_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    bsa_kernel<true><<<items, kBsaThreads, smem, stream>>>(maps, batch, args);
-  } else {
-    e = cudaFuncSetAttribute(bsa_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    bsa_kernel<false><<<items, kBsaThreads, smem, stream>>>(maps, batch, args);
-  }
-  return cudaGetLastError();
+  if (args.block != kBlock && args.block != kHalf) return cudaErrorInvalidValue;
+  const bool b64 = args.block == kHalf;
+  return fp8 ? (b64 ? launch_bsa_t<true, true>(maps, batch, args, items, stream)
+                    : launch_bsa_t<true, false>(maps, batch, args, items, stream))
+             : (b64 ? launch_bsa_t<false, true>(maps, batch, args, items, stream)
+                    : launch_bsa_t<false, false>(maps, batch, args, items, stream));
 }
 
 }  // namespace stem

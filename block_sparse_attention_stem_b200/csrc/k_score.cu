@@ -61,7 +61,7 @@ struct ScoreSmem {
 
 }  // namespace
 
-template <bool kFp8, int kS>
+template <bool kFp8, int kS, int kB>
 __global__ void __launch_bounds__(kScoreThreads, 1)
     score_kernel(const __grid_constant__ ScoreMaps maps, const SeqBatch batch, const ScoreArgs args) {
   extern __shared__ uint8_t smem_raw[];
@@ -71,9 +71,11 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
   const int seq = find_seq(batch, blockIdx.x);
   const int local = blockIdx.x - batch.item0[seq];
   constexpr int s = kS;  // scoring stride (compile-time so the pooling indices are)
+  constexpr int gpb = kB / s;                      // groups per block (16 for 128-token blocks, s = 8)
+  constexpr int kBlocksPerTile = kTileM / gpb;     // query blocks per 128-group query tile
   const int nb = batch.nb[seq];
   const int L = batch.len[seq];
-  const int ntile = (nb + s - 1) / s;  // query tiles of 128 groups = s blocks
+  const int ntile = (nb + kBlocksPerTile - 1) / kBlocksPerTile;
   // KV heads in groups of g; inside a group, query tiles descending (query
   // tile, KV head, head pair of the group).  A CTA's work grows with its
   // query tile.  When one KV head's CTAs outnumber the SMs, g = 1: the CTAs in
@@ -237,7 +239,6 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     const int h = h0 + e;
     const int q4 = warp & 3;
     const int row = q4 * 32 + lane;
-    constexpr int gpb = kBlock / s;             // groups per block (16 for s = 8)
     const int a = I * kTileM + row;              // query group within the sequence
     const bool row_valid = a * s < L;
     const int i = a / gpb;                       // query block (local)
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
     float* srow = args.scores + (static_cast<size_t>(h) * args.nbtot + g) * args.nb_max;
     const bool writer = (lane % gpb) == 0 && row_valid && i < nb;
     const float ninf = -__int_as_float(0x7f800000);
-    constexpr int kbt = kTileN / gpb;    // key blocks per key tile (2 s)
+    constexpr int kbt = kTileN / gpb;    // key blocks per key tile (at most 32: one per lane)
     constexpr int kbc = 32 / gpb;        // key blocks per 32-column chunk
     constexpr int kbh = kbt / 2;         // key blocks per half tile
     bool complete = true;
@@ -356,15 +357,22 @@ __global__ void __launch_bounds__(kScoreThreads, 1)
 
 size_t score_smem_bytes() { return sizeof(ScoreSmem) + 1024; }
 
-template <bool kFp8, int kS>
+template <bool kFp8, int kS, int kB>
 static cudaError_t launch_score_t(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args,
                                   cudaStream_t stream) {
   const size_t smem = score_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(score_kernel<kFp8, kS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(score_kernel<kFp8, kS, kB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  score_kernel<kFp8, kS><<<batch.item0[batch.n], kScoreThreads, smem, stream>>>(maps, batch, args);
+  score_kernel<kFp8, kS, kB><<<batch.item0[batch.n], kScoreThreads, smem, stream>>>(maps, batch, args);
   return cudaGetLastError();
+}
+
+template <int kS, int kB>
+static cudaError_t launch_score_b(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args, bool fp8,
+                                  cudaStream_t stream) {
+  return fp8 ? launch_score_t<true, kS, kB>(maps, batch, args, stream)
+             : launch_score_t<false, kS, kB>(maps, batch, args, stream);
 }
 
 cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const ScoreArgs& args_in, bool fp8,
@@ -375,10 +383,12 @@ cudaError_t launch_score(const ScoreMaps& maps, const SeqBatch& batch, const Sco
   cudaError_t e = cudaGetDevice(&dev);
   if (e == cudaSuccess) e = cudaDeviceGetAttribute(&args.num_sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
+  const bool b64 = args.block == kBlock / 2;
+  if (!b64 && args.block != kBlock) return cudaErrorInvalidValue;
   if (args.stride == 8)
-    return fp8 ? launch_score_t<true, 8>(maps, batch, args, stream) : launch_score_t<false, 8>(maps, batch, args, stream);
+    return b64 ? launch_score_b<8, 64>(maps, batch, args, fp8, stream) : launch_score_b<8, 128>(maps, batch, args, fp8, stream);
   if (args.stride == 4)
-    return fp8 ? launch_score_t<true, 4>(maps, batch, args, stream) : launch_score_t<false, 4>(maps, batch, args, stream);
+    return b64 ? launch_score_b<4, 64>(maps, batch, args, fp8, stream) : launch_score_b<4, 128>(maps, batch, args, fp8, stream);
   return cudaErrorInvalidValue;
 }
 

@@ -5,8 +5,8 @@
 //   vbonus[hk][g0 + j] = beta * max(0, ln max_{t in block j} ||v_t||^2)
 //
 // Two CTAs per key block, each taking half of the KV heads, read the block's
-// 128 tokens x Hkv heads x 128 values (256 KB bf16 in the packed [T, Hkv, d]
-// layout; each CTA reads 1 KB of every 2 KB token row) once with 16-byte
+// 128 (or 64) tokens x Hkv heads x 128 values (256 KB bf16 in the packed
+// [T, Hkv, d] layout; each CTA reads 1 KB of every 2 KB token row) once with 16-byte
 // loads; 16 (bf16) or 8 (fp8) lanes cover one (token, head) row of 128
 // values, and each thread keeps eight rows' loads in flight.  Measured at
 // 8 KV heads (one launch each, cold L2): with four rows in flight and one CTA
@@ -27,16 +27,16 @@ namespace stem {
 template <bool kFp8>
 __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const uint8_t* __restrict__ v,
                                                     const float* __restrict__ v_scale, int hkv, int hk_first,
-                                                    int nhk_all, int heads_per_cta, int nbtot, float beta,
-                                                    bool raw_log, float* __restrict__ vbonus) {
+                                                    int nhk_all, int heads_per_cta, int nbtot, int block,
+                                                    float beta, bool raw_log, float* __restrict__ vbonus) {
   extern __shared__ unsigned int s_max[];  // [nhk] bit patterns of non-negative floats (KV heads hk0 ..)
   // this CTA's KV heads: hk0 .. hk0 + nhk - 1 (group blockIdx.y of the launch's range)
   const int hk0 = hk_first + static_cast<int>(blockIdx.y) * heads_per_cta;
   const int nhk = min(heads_per_cta, hk_first + nhk_all - hk0);
   const int s = find_seq(batch, blockIdx.x);
   const int j = blockIdx.x - batch.item0[s];
-  const int t0 = j * kBlock;
-  const int ntok = min(kBlock, batch.len[s] - t0);
+  const int t0 = j * block;
+  const int ntok = min(block, batch.len[s] - t0);
   for (int h = threadIdx.x; h < nhk; h += blockDim.x) s_max[h] = 0u;
   __syncthreads();
 
@@ -117,7 +117,8 @@ __global__ void __launch_bounds__(256) vnorm_kernel(const SeqBatch batch, const 
 }
 
 cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
-                         int nhk, int nbtot, float beta, bool raw_log, float* vbonus, cudaStream_t stream) {
+                         int nhk, int nbtot, int block, float beta, bool raw_log, float* vbonus,
+                         cudaStream_t stream) {
   const int items = batch.item0[batch.n];
   if (items == 0 || nhk <= 0) return cudaSuccess;
   const int heads_per_cta = (nhk + 1) / 2;  // two head groups (one when nhk = 1)
@@ -125,10 +126,10 @@ cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_sc
   const size_t smem = sizeof(unsigned int) * static_cast<size_t>(heads_per_cta);
   if (fp8)
     vnorm_kernel<true><<<grid, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                    heads_per_cta, nbtot, beta, raw_log, vbonus);
+                                                    heads_per_cta, nbtot, block, beta, raw_log, vbonus);
   else
     vnorm_kernel<false><<<grid, 256, smem, stream>>>(batch, static_cast<const uint8_t*>(v), v_scale, hkv, hk0, nhk,
-                                                     heads_per_cta, nbtot, beta, raw_log, vbonus);
+                                                     heads_per_cta, nbtot, block, beta, raw_log, vbonus);
   return cudaGetLastError();
 }
 

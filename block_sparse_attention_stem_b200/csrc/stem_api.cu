@@ -45,6 +45,7 @@ struct SeqInfo {
 struct Plan {
   stem_plan_t pub;
   std::vector<SeqInfo> seqs;  // non-empty sequences, longest first
+  int B = kBlock;             // block size (tokens): 128, or 64
   size_t off_vbonus, off_vwide, off_scores, off_budgets, off_rowptr, off_colidx;
 };
 
@@ -60,8 +61,9 @@ stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
   for (int s = 0; s < qkv->num_seqs; ++s)
     if (cu[s + 1] < cu[s]) return STEM_ERR_INVALID_ARG;
   if (cu[qkv->num_seqs] != qkv->total_tokens) return STEM_ERR_INVALID_ARG;
-  if (p->block_size != kBlock) return p->block_size < 1 ? STEM_ERR_INVALID_ARG : STEM_ERR_UNSUPPORTED;
-  if (p->stride < 1 || kBlock % p->stride != 0) return STEM_ERR_INVALID_ARG;
+  if (p->block_size != kBlock && p->block_size != kBlock / 2)
+    return p->block_size < 1 ? STEM_ERR_INVALID_ARG : STEM_ERR_UNSUPPORTED;
+  if (p->stride < 1 || p->block_size % p->stride != 0) return STEM_ERR_INVALID_ARG;
   if (p->stride != 4 && p->stride != 8) return STEM_ERR_UNSUPPORTED;
   if (p->chunk_size < 1) return STEM_ERR_INVALID_ARG;
   if (!(p->norm > 0.0) || !std::isfinite(p->norm)) return STEM_ERR_INVALID_ARG;
@@ -80,23 +82,24 @@ stem_status_t make_plan(const stem_qkv_t* qkv, const stem_params_t* p, Plan* out
   stem_status_t st = validate(qkv, p);
   if (st != STEM_OK) return st;
   const int hq = qkv->num_q_heads, hkv = qkv->num_kv_heads;
-  const int s = p->stride, gpb = kBlock / s;
+  const int s = p->stride, B = p->block_size, gpb = B / s;
   Plan pl{};
+  pl.B = B;
   int64_t nbtot = 0, nb_max = 0, nnz_h = 0;
   double pairs_sel = 0, pairs_dense = 0, score_pairs = 0;
   for (int q = 0; q < qkv->num_seqs; ++q) {
     const int32_t o = qkv->cu_seqlens_host[q];
     const int32_t L = qkv->cu_seqlens_host[q + 1] - o;
-    const int32_t nb = (L + kBlock - 1) / kBlock;
+    const int32_t nb = (L + B - 1) / B;
     if (nb > 0) {
       SeqInfo si{q, o, L, nb, static_cast<int32_t>(nbtot), nnz_h};
       for (int i = 0; i < nb; ++i) {
         const int32_t b = tpd_budget(i, nb, p->keep_ratio, p->mu, p->sink_blocks, p->window_blocks,
                                      p->budget_mode);
         nnz_h += b;
-        const double qi = std::min(kBlock, L - i * kBlock);
-        pairs_sel += (b - 1) * qi * kBlock + qi * (qi + 1) / 2;
-        pairs_dense += static_cast<double>(i) * qi * kBlock + qi * (qi + 1) / 2;
+        const double qi = std::min(B, L - i * B);
+        pairs_sel += (b - 1) * qi * B + qi * (qi + 1) / 2;
+        pairs_dense += static_cast<double>(i) * qi * B + qi * (qi + 1) / 2;
       }
       score_pairs += static_cast<double>(nb) * (nb + 1) / 2 * gpb * gpb;
       pl.seqs.push_back(si);
@@ -105,6 +108,9 @@ stem_status_t make_plan(const stem_qkv_t* qkv, const stem_params_t* p, Plan* out
     nb_max = std::max<int64_t>(nb_max, nb);
   }
   if (nb_max == 0) nb_max = 1;
+  // 64-token blocks: the attention keeps each pair of lists as two bitmaps of
+  // kMaxBitmapBlocks bits in shared memory
+  if (B != kBlock && nb_max > kMaxBitmapBlocks) return STEM_ERR_UNSUPPORTED;
   const int64_t rows = static_cast<int64_t>(hq) * nbtot;
   const int64_t nnz = nnz_h * hq;
   if (nnz > INT32_MAX || rows + 1 > INT32_MAX) return STEM_ERR_UNSUPPORTED;
@@ -252,7 +258,7 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   const int nbtot = static_cast<int>(pl.pub.nb_total), nb_max = static_cast<int>(pl.pub.nb_max);
   for (const SeqBatch& b : make_batches(pl, [](const SeqInfo& si) { return si.nb; })) {
     stem_status_t st = cuda_status(
-        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, hk0, nhk, nbtot, static_cast<float>(p->beta),
+        launch_vnorm(b, qkv->v, qkv->v_scale, fp8, hkv, hk0, nhk, nbtot, pl.B, static_cast<float>(p->beta),
                      p->bonus_mode == STEM_BONUS_STANDARDIZED, vbonus, stream));
     if (st != STEM_OK) return st;
   }
@@ -268,6 +274,7 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   a.nbtot = nbtot;
   a.nb_max = nb_max;
   a.stride = s;
+  a.block = pl.B;
   a.scale = static_cast<float>(1.0 / (std::sqrt(static_cast<double>(kHeadDim)) * s * p->norm));
   a.q_scale = qkv->q_scale;
   a.k_scale = qkv->k_scale;
@@ -281,9 +288,13 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
   a.budgets = budgets;
   a.row_ptr = row_ptr;
   a.col_idx = col_idx;
-  // one CTA per (pair of query heads of a KV group, 128-group query tile)
+  // one CTA per (pair of query heads of a KV group, 128-group query tile of
+  // 128 s / B query blocks)
   const int pairs = nhk * ((hq / hkv + 1) / 2);
-  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) { return pairs * ((si.nb + s - 1) / s); })) {
+  const int blocks_per_tile = 128 * s / pl.B;
+  for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) {
+         return pairs * ((si.nb + blocks_per_tile - 1) / blocks_per_tile);
+       })) {
     ScoreMaps maps;
     std::memset(&maps, 0, sizeof(maps));
     for (int q = 0; q < b.n; ++q) {
@@ -371,6 +382,7 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
   a.lse = lse;
   a.status = status;
   a.hk0 = hk0;
+  a.block = pl.B;
   BsaMaps maps;
   std::memset(&maps, 0, sizeof(maps));
   if (paged) {
@@ -384,11 +396,14 @@ stem_status_t run_bsa(const stem_qkv_t* qkv, const stem_params_t* p, const Plan&
     a.max_pages = paged->max_pages_per_seq;
   }
   // one CTA per CSR row (query head, query block), or, with lists shared by
-  // the query heads of a group, per (query block, pair of query heads)
+  // the query heads of a group, per (query block, pair of query heads); with
+  // 64-token blocks one CTA per query head and pair of query blocks (one
+  // 128-token query tile)
   const int G = hq / hkv;
-  const bool pairs = p->list_mode == STEM_LIST_PER_GROUP && G >= 2;
+  const bool pairs = p->list_mode == STEM_LIST_PER_GROUP && G >= 2 && pl.B == kBlock;
   for (const SeqBatch& b : make_batches(pl, [&](const SeqInfo& si) {
-         return pairs ? nhk * ((G + 1) / 2) * si.nb : nhk * G * si.nb;
+         const int tiles = pl.B == kBlock ? si.nb : (si.nb + 1) / 2;
+         return pairs ? nhk * ((G + 1) / 2) * tiles : nhk * G * tiles;
        })) {
     for (int q = 0; q < b.n; ++q) {
       // Q in 128-token boxes; K and V in 64-token boxes (the attention
@@ -508,8 +523,8 @@ stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_paged_kv_t* k
   if (static_cast<int64_t>(kv->num_pages) * kv->page_size > INT32_MAX) return STEM_ERR_INVALID_ARG;
   for (int q = 0; q < qkv->num_seqs; ++q) {
     const int64_t L = qkv->cu_seqlens_host[q + 1] - qkv->cu_seqlens_host[q];
-    // the last key block may run past L to its 128-token end
-    const int64_t need = (L + kBlock - 1) / kBlock * kBlock;
+    // the last key block may run past L to its end (a multiple of the block size)
+    const int64_t need = (L + params->block_size - 1) / params->block_size * params->block_size;
     if (need > static_cast<int64_t>(kv->max_pages_per_seq) * kv->page_size) return STEM_ERR_INVALID_ARG;
   }
   if (!row_ptr || !col_idx || !out || !lse || !ws) return STEM_ERR_INVALID_ARG;

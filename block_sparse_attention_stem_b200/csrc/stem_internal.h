@@ -18,7 +18,8 @@ namespace stem {
 constexpr int STEM_ERR_TIMEOUT_CODE = 6;
 constexpr int STEM_ERR_BAD_BLOCKLIST_CODE = 7;
 
-constexpr int kBlock = 128;      // attention block (tokens)
+constexpr int kBlock = 128;      // block (tokens); also the attention's query tile for 64-token blocks
+constexpr int kMaxBitmapBlocks = 32768;  // 64-token blocks: longest sequence in blocks (2,097,152 tokens)
 constexpr int kHeadDim = 128;    // supported head_dim
 constexpr int kMaxSeqPerLaunch = 8;
 

@@ -32,6 +32,7 @@ struct BsaMaps {
 
 struct ScoreArgs {
   int hq, hkv, nbtot, nb_max, stride;
+  int block;                // block size (tokens): 128 or 64
   int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
   int num_sms;              // SMs of the device (the CTA order depends on it, never the results)
   float scale;              // 1 / (sqrt(d) s n)
@@ -54,6 +55,7 @@ constexpr int kFusedSelectMaxBlocks = 5888;
 
 struct BsaArgs {
   int hq, hkv, nbtot, total_tokens;
+  int block;                // block size (tokens): 128, or 64 (one CTA then covers query blocks 2p and 2p + 1)
   int hk0;                  // first KV head of the launch (its items cover consecutive KV heads)
   const int32_t* page_table;  // paged K/V: [num_seqs][max_pages] physical page per logical page, else null
   int page_size;            // tokens per page, a multiple of 64
@@ -73,7 +75,8 @@ struct BsaArgs {
 // KV heads hk0 .. hk0 + nhk - 1 only.  raw_log: write x = ln max ||v||^2 for a
 // later launch_bonus_standardize instead of beta * max(0, x).
 cudaError_t launch_vnorm(const SeqBatch& batch, const void* v, const float* v_scale, bool fp8, int hkv, int hk0,
-                         int nhk, int nbtot, float beta, bool raw_log, float* vbonus, cudaStream_t stream);
+                         int nhk, int nbtot, int block, float beta, bool raw_log, float* vbonus,
+                         cudaStream_t stream);
 // vbonus[hk][g] = beta * max(0, (x - mean) / std) over the finite x of each
 // sequence, for KV heads hk0 .. hk0 + (items per sequence) - 1.
 cudaError_t launch_bonus_standardize(const SeqBatch& batch, int hk0, int nbtot, float beta, float* vbonus,

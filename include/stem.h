@@ -94,7 +94,10 @@ typedef enum {
 
 /* Method parameters (AngelSlim documentation §6 defaults in brackets). */
 typedef struct {
-  int32_t block_size;     /* attention block [128]; only 128 is supported */
+  int32_t block_size;     /* block of the scores, lists and attention [128]: 128 or 64 (the
+                             "64x128 or 128x128" KV blocks of the HPC-BSA article §3.1);
+                             with 64, sequences of at most 2,097,152 tokens
+                             (STEM_ERR_UNSUPPORTED beyond) */
   int32_t stride;         /* scoring downsampling stride s [8]; 4 or 8 are supported */
   int32_t chunk_size;     /* scoring query-chunk width [2048]; > 0; does not change results */
   double  norm;           /* extra scoring normalisation n [1.0]; > 0 */
@@ -240,7 +243,8 @@ STEM_API stem_status_t stem_bsa_fwd(const stem_qkv_t* qkv, const stem_params_t* 
  * not used and may be NULL; q, cu_seqlens and the fp8 scales as for
  * stem_bsa_fwd).  Results equal stem_bsa_fwd's on the packed K/V the pages
  * hold, bit for bit.  Page rows past a sequence's last token (up to its next
- * multiple of 128) are read: they must hold finite values, zeros for example.
+ * multiple of the block size) are read: they must hold finite values, zeros
+ * for example.
  * A page number outside [0, num_pages) reads zeros.  STEM_ERR_INVALID_ARG for
  * a page size that is not a positive multiple of 64 or a table too short for
  * some sequence. */

@@ -87,13 +87,32 @@ def test_plan_density_of_the_128k_workload():
 
 @pytest.mark.parametrize("rho,mu,mode,S,W", [(0.3, 0.45, 0, 4, 4), (0.1, 1.0, 0, 0, 1), (0.25, 0.7, 1, 1, 2),
                                              (1.0, 1.0, 0, 0, 1), (0.05, 0.2, 1, 3, 5)])
-def test_plan_budgets_equal_oracle_on_odd_parameters(rho, mu, mode, S, W):
+@pytest.mark.parametrize("B", [128, 64])
+def test_plan_budgets_equal_oracle_on_odd_parameters(rho, mu, mode, S, W, B):
     seqlens = [12800, 1000, 129, 1]
     qkv = fake_qkv(seqlens, 4, 2)
-    p = dict(keep_ratio=rho, mu=mu, budget_mode=mode, sink_blocks=S, window_blocks=W)
+    p = dict(keep_ratio=rho, mu=mu, budget_mode=mode, sink_blocks=S, window_blocks=W, block_size=B)
     pl = b.stem_plan(qkv, b.make_params(**p))
     bud = O.budgets([0] + list(np.cumsum(seqlens)), O.Params(**p))
     assert pl.nnz_per_head == int(bud.sum())
+    assert pl.nb_total == sum(math.ceil(L / B) for L in seqlens) == len(bud)
+    assert pl.nb_max == math.ceil(max(seqlens) / B)
+    # score FLOPs: 2 s d Hq sum NB(NB+1)/2 (B/s)^2
+    pairs = sum(math.ceil(L / B) * (math.ceil(L / B) + 1) // 2 for L in seqlens)
+    assert pl.score_flops == pytest.approx(2 * 8 * 128 * 4 * pairs * (B // 8) ** 2)
+
+
+def test_plan_rejects_64_token_blocks_past_the_bitmap_limit():
+    # 64-token blocks keep each tile's two lists as bitmaps of 32768 blocks;
+    # planning reads only the host offsets, so one-token tensors stand in
+    t = torch.zeros(1, 2, 128, dtype=torch.bfloat16)
+
+    def qkv(L):
+        return b.make_qkv(t, t, t, [0, L], cu_seqlens_dev=torch.zeros(1))
+
+    assert b.stem_plan(qkv(32768 * 64), b.make_params(block_size=64)).nb_max == 32768
+    assert _status(lambda: b.stem_plan(qkv(32768 * 64 + 1), b.make_params(block_size=64))) == 2
+    assert b.stem_plan(qkv(32768 * 64 + 1), b.make_params(block_size=128)).nb_max == 16385
 
 
 def _status(fn):
@@ -122,7 +141,12 @@ def test_validation_rejects_bad_parameters():
     b.stem_plan(qkv, P(list_mode=1))  # GQA-shared lists are valid
     assert _status(lambda: b.stem_plan(qkv, P(stride=3))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(stride=16))) == 2
-    assert _status(lambda: b.stem_plan(qkv, P(block_size=64))) == 2
+    b.stem_plan(qkv, P(block_size=64))  # 64-token blocks are valid
+    assert _status(lambda: b.stem_plan(qkv, P(block_size=32))) == 2
+    assert _status(lambda: b.stem_plan(qkv, P(block_size=96))) == 2
+    assert _status(lambda: b.stem_plan(qkv, P(block_size=0))) == 1
+    assert _status(lambda: b.stem_plan(qkv, P(block_size=64, stride=16))) == 2  # divides 64, not supported
+    assert _status(lambda: b.stem_plan(qkv, P(block_size=64, stride=3))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(norm=float("nan")))) == 1
 
 

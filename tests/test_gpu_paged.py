@@ -53,6 +53,9 @@ CASES = {
     "gqa_page128": (W([1500, 700], 6, 2, seed=51), 128),
     "fp8_page256": (W([640, 2048, 77], 4, 2, dtype="fp8", seed=52), 256),
     "shared_lists_page64": (W([1000, 128, 2088], 8, 2, seed=53, list_mode=1), 64),  # two heads per CTA
+    # 64-token blocks: every 64-key unit is one page lookup
+    "b64_page64": (W([1000, 128, 2088, 63], 8, 2, seed=54, block_size=64), 64),
+    "b64_fp8_page128": (W([640, 2112, 77], 4, 2, dtype="fp8", seed=55, block_size=64), 128),
 }
 
 
@@ -77,7 +80,7 @@ def test_paged_equals_packed(name):
     assert torch.equal(lse.view(torch.int32), lse_ref.view(torch.int32))
 
 
-@pytest.mark.parametrize("name", ["varlen_page64", "fp8_page256"])
+@pytest.mark.parametrize("name", ["varlen_page64", "fp8_page256", "b64_page64", "b64_fp8_page128"])
 def test_paged_attention_matches_oracle_through_the_gather(name):
     w, ps = CASES[name]
     cu = w.cu_seqlens()

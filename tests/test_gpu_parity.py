@@ -52,6 +52,16 @@ CASES = {
     "group_lists": W([1000, 128, 2088], 8, 2, seed=21, list_mode=1),
     "group_lists_odd_group": W([1500, 700], 6, 2, seed=22, list_mode=1, keep_ratio=0.25),
     "group_lists_fp8": W([640, 2048, 77], 4, 2, dtype="fp8", seed=23, list_mode=1),
+    # 64-token blocks ("64x128" KV blocks): the attention's 128-row tile holds
+    # query blocks 2p and 2p + 1 and walks the union of their lists; odd block
+    # counts (2088 -> 33, 63 -> 1) leave a last tile with one query block
+    "b64_varlen": W([1000, 128, 2088, 64, 63], 8, 2, seed=31, block_size=64, sink_blocks=2, window_blocks=2),
+    "b64_fp8": W([640, 2112, 77], 4, 2, dtype="fp8", seed=32, block_size=64),
+    "b64_stride4": W([1600], 2, 1, seed=33, stride=4, block_size=64, keep_ratio=0.3),
+    "b64_multi_tile": W([4096 + 640 + 64], 4, 2, seed=34, keep_ratio=0.3, block_size=64, sink_blocks=1,
+                        window_blocks=1),
+    "b64_group_lists": W([1000, 2088], 8, 2, seed=35, list_mode=1, block_size=64),
+    "b64_std_bonus_fp8": W([640, 2112, 77], 4, 2, dtype="fp8", seed=36, bonus_mode=1, block_size=64),
 }
 
 
@@ -68,7 +78,7 @@ class Case:
         self.p = oparams(w)
         self.q, self.k, self.v = oracle_arrays(self.inp, w.dtype)
         self.ref_scores = O.block_scores(self.q, self.k, self.v, self.cu, self.p)
-        self.ref_bonus = O.value_bonus(self.v, self.cu, self.p.beta, mode=self.p.bonus_mode)
+        self.ref_bonus = O.value_bonus(self.v, self.cu, self.p.beta, self.p.block_size, mode=self.p.bonus_mode)
 
 
 _cache = {}
@@ -85,7 +95,7 @@ def test_scores_and_bonus(name):
     c = get_case(name)
     scores, vbonus, ws = b.stem_score(c.qkv, c.params)
     assert b.stem_read_device_status(ws) == 0
-    check_scores(scores.cpu().numpy().astype(np.float64), c.ref_scores, c.cu)
+    check_scores(scores.cpu().numpy().astype(np.float64), c.ref_scores, c.cu, c.p.block_size)
     vb = vbonus.cpu().numpy().astype(np.float64)
     np.testing.assert_allclose(vb, c.ref_bonus, rtol=1e-5, atol=1e-5)
 
@@ -182,7 +192,8 @@ def test_prefill_end_to_end(name):
     rp, ci = rp.cpu().numpy(), ci.cpu().numpy()
     ob, orp, oci = O.select(c.ref_scores, c.cu, c.p, hkv=c.w.num_kv_heads)
     ranked = O.group_pooled_scores(c.ref_scores, c.w.num_kv_heads) if c.p.list_mode else c.ref_scores
-    compare_lists(rp, ci, orp, oci, ranked, c.cu, c.w.num_q_heads, c.p.sink_blocks, c.p.window_blocks)
+    compare_lists(rp, ci, orp, oci, ranked, c.cu, c.w.num_q_heads, c.p.sink_blocks, c.p.window_blocks,
+                  c.p.block_size)
     # attention with the GPU's own lists
     ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp, ci, c.p)
     check_attention(out, lse, ro, rl, c.w.dtype)
@@ -194,11 +205,11 @@ def test_prefill_end_to_end(name):
     assert torch.equal(out2, out) and torch.equal(lse2, lse)
 
 
-@pytest.mark.parametrize("name", ["tiny", "varlen", "varlen_fp8", "multi_tile"])
+@pytest.mark.parametrize("name", ["tiny", "varlen", "varlen_fp8", "multi_tile", "b64_varlen", "b64_fp8"])
 def test_dense_comparator_is_causal_attention(name):
     """Every causal block listed: the result is ordinary causal attention."""
     c = get_case(name)
-    rp, ci = O.full_csr(c.cu, c.w.num_q_heads)
+    rp, ci = O.full_csr(c.cu, c.w.num_q_heads, c.p.block_size)
     out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, torch.from_numpy(rp.astype(np.int32)).cuda(),
                                   torch.from_numpy(ci.astype(np.int32)).cuda())
     assert b.stem_read_device_status(ws) == 0
@@ -225,9 +236,30 @@ def test_malformed_list_entries_are_skipped_and_reported():
     check_attention(out, lse, ro, rl, "bf16")
 
 
-def test_empty_rows_give_zero_output_and_minus_inf_lse():
-    c = get_case("tiny")
-    nrows = 2 * 16
+def test_malformed_list_entries_are_skipped_and_reported_64_token_blocks():
+    """With 64-token blocks the bad entry sits in the second list of a tile
+    (query block 7 = rows 64-127 of the tile of blocks 6 and 7)."""
+    c = get_case("b64_varlen")
+    rp, ci = O.full_csr(c.cu, c.w.num_q_heads, 64)
+    seqs, nbtot = O.seq_blocks(c.cu, 64)
+    r = 1 * nbtot + 7
+    bad = ci.copy()
+    bad[rp[r] + 2] = 9  # above the diagonal
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, torch.from_numpy(rp.astype(np.int32)).cuda(),
+                                  torch.from_numpy(bad.astype(np.int32)).cuda())
+    assert b.stem_read_device_status(ws) == 7
+    keep = np.ones(len(ci), dtype=bool)
+    keep[rp[r] + 2] = False
+    rp2 = rp.copy()
+    rp2[r + 1:] -= 1
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp2, ci[keep], c.p)
+    check_attention(out, lse, ro, rl, "bf16")
+
+
+@pytest.mark.parametrize("name", ["tiny", "b64_varlen"])
+def test_empty_rows_give_zero_output_and_minus_inf_lse(name):
+    c = get_case(name)
+    nrows = c.w.num_q_heads * O.seq_blocks(c.cu, c.p.block_size)[1]
     rp = torch.zeros(nrows + 1, dtype=torch.int32, device="cuda")
     ci = torch.zeros(1, dtype=torch.int32, device="cuda")
     out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, rp, ci)

@@ -433,6 +433,70 @@ def test_beta_zero_is_pure_routing():
             assert S0[0, i, j] == D[i * 4:(i + 1) * 4, j * 4:(j + 1) * 4].max()
 
 
+def test_halving_the_block_refines_scores_and_bonus():
+    """64x128 or 128x128 KV blocks (HPC-BSA article §3.1): with beta = 0 an
+    off-diagonal score at block size B is the max of the four block-size-B/2
+    scores it covers (both are maxima of the same downsampled entries), and the
+    value bonus at B is the larger of its two halves' bonuses (the max over a
+    union of tokens, then the monotone ln and max(0, .))."""
+    rng = np.random.default_rng(21)
+    B, s, d = 16, 4, 8
+    L = 9 * B + 5  # ragged last block at both sizes
+    q, k = rng.standard_normal((L, 2, d)), rng.standard_normal((L, 1, d))
+    v = rng.standard_normal((L, 1, d)) * np.exp(rng.standard_normal((L, 1, 1)))
+    S = O.block_scores(q, k, v, [0, L], O.Params(block_size=B, stride=s, beta=0.0))
+    Sh = O.block_scores(q, k, v, [0, L], O.Params(block_size=B // 2, stride=s, beta=0.0))
+    nb, nbh = S.shape[1], Sh.shape[1]
+    assert nbh == O.cdiv(L, B // 2) and nb == O.cdiv(L, B)
+    for h in range(2):
+        for i in range(nb):
+            for j in range(i):
+                sub = [Sh[h, a, c] for a in (2 * i, 2 * i + 1) if a < nbh for c in (2 * j, 2 * j + 1)]
+                assert S[h, i, j] == max(sub)
+            # the diagonal also covers the sub-block above the half-size diagonal
+            diag_sub = [Sh[h, a, c] for a in (2 * i, 2 * i + 1) if a < nbh for c in (2 * i, 2 * i + 1) if c <= a]
+            assert S[h, i, i] >= max(diag_sub)
+    bon = O.value_bonus(v, [0, L], 0.3, B)[0]
+    bonh = O.value_bonus(v, [0, L], 0.3, B // 2)[0]
+    for j in range(nb):
+        assert bon[j] == max(bonh[2 * j:2 * j + 2])
+
+
+def test_attention_with_refined_lists_equals_the_coarse_attention():
+    """A list at block size B, refined to block size B/2 (both halves of every
+    listed block, for both half-size query blocks), keeps the same causal key
+    set for every query, so the attention is the same."""
+    B, d = 16, 8
+    seqlens = [7 * B + 3, 2 * B, 5]
+    q, k, v, cu = _small_problem(seqlens, 4, 2, d, seed=23)
+    rng = np.random.default_rng(24)
+    p = O.Params(block_size=B)
+    ph = O.Params(block_size=B // 2)
+    seqs, nbtot = O.seq_blocks(cu, B)
+    seqsh, nbtoth = O.seq_blocks(cu, B // 2)
+    rows, rowsh = [], [[] for _ in range(4 * nbtoth)]
+    for h in range(4):
+        for (o, L, nb, g0), (_, _, nbh, g0h) in zip(seqs, seqsh):
+            for i in range(nb):
+                lst = sorted(set(rng.choice(i + 1, size=rng.integers(1, i + 2), replace=False).tolist()) | {i})
+                rows.append(lst)
+                for a in (2 * i, 2 * i + 1):
+                    if a < nbh:
+                        rowsh[h * nbtoth + g0h + a] = [c for j in lst for c in (2 * j, 2 * j + 1) if c <= a]
+
+    def csr(rs):
+        rp = np.zeros(len(rs) + 1, dtype=np.int64)
+        rp[1:] = np.cumsum([len(r) for r in rs])
+        return rp, np.array([j for r in rs for j in r], dtype=np.int64)
+
+    rp, ci = csr(rows)
+    rph, cih = csr(rowsh)
+    O1, L1 = O.bsa(q, k, v, cu, rp, ci, p)
+    O2, L2 = O.bsa(q, k, v, cu, rph, cih, ph)
+    np.testing.assert_allclose(O2, O1, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(L2, L1, rtol=0, atol=1e-12)
+
+
 # ---------------------------------------------------------------- attention
 
 def _small_problem(seqlens, hq, hkv, d, seed):
