@@ -60,7 +60,7 @@ def parse_args(argv=None):
     ap.add_argument("--mode", choices=["default", "sweep", "fp8stack", "quality", "variants", "once"], default="default",
                     help="sweep: latency vs kept-block density (64K, mu=1); fp8stack: the 36-layer fp8 varlen stack; "
                          "quality: reconstruction error against dense attention (32K); "
-                         "variants: the 128K step with the standardized bonus and KV-group-shared lists; "
+                         "variants: the 128K step with the standardized bonus, KV-group-shared lists and 64-token blocks; "
                          "once: one untimed step of --workload (the command profilers wrap)")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
     ap.add_argument("--separate-select", action="store_true",
@@ -767,8 +767,9 @@ def run_quality(args):
 
 def run_variants(args):
     """The step on the 128K workload with the selection variants beside the
-    default: the standardized value bonus (bonus_mode 1) and KV-group-shared
-    block lists (list_mode 1); ms per stage and attention TFLOP/s."""
+    default: the standardized value bonus (bonus_mode 1), KV-group-shared
+    block lists (list_mode 1) and 64-token blocks (block_size 64, 2048 blocks
+    per row); ms per stage and attention TFLOP/s."""
     import torch
     from block_sparse_attention_stem_b200 import binding as b
     from block_sparse_attention_stem_b200 import inputs as I
@@ -781,7 +782,8 @@ def run_variants(args):
     sampler.start()
     for label, kw in (("default (log bonus, per-head lists)", {}),
                       ("standardized bonus (bonus_mode 1)", dict(bonus_mode=1)),
-                      ("KV-group-shared lists (list_mode 1)", dict(list_mode=1))):
+                      ("KV-group-shared lists (list_mode 1)", dict(list_mode=1)),
+                      ("64-token blocks (block_size 64)", dict(block_size=64))):
         params = b.make_params(**dict(w0.params(), **kw))
         pl = b.stem_plan(qkv, params)
         st = {}

@@ -91,7 +91,7 @@ def _check_every_row(w, inp, res):
     (a swapped pair's oracle scores within TIE_REL), forced blocks present."""
     p = O.Params(**w.params())
     cu = w.cu_seqlens()
-    seqs, nbtot = O.seq_blocks(cu)
+    seqs, nbtot = O.seq_blocks(cu, p.block_size)
     G = w.num_q_heads // w.num_kv_heads
     rp = res["row_ptr"].cpu().numpy().astype(np.int64)
     ci = res["col_idx"].cpu().numpy().astype(np.int64)
@@ -140,7 +140,8 @@ def _check_workload(w, samples, every_row=False):
     inp, qkv, res = _run(w)
     p = O.Params(**w.params())
     cu = w.cu_seqlens()
-    seqs, nbtot = O.seq_blocks(cu)
+    B = p.block_size
+    seqs, nbtot = O.seq_blocks(cu, B)
     hq = w.num_q_heads
     # --- every row: budgets, row pointers, list structure
     bud = O.budgets(cu, p)
@@ -200,7 +201,7 @@ def _check_workload(w, samples, every_row=False):
         rp1 = np.zeros(nb + 1, dtype=np.int64)
         rp1[i + 1:] = len(G_list)
         ro, rl = O.bsa(qh, kh, vh, [0, L], rp1, G_list, p, rows_subset=[(0, i)])
-        t0, t1 = i * 128, min((i + 1) * 128, L)
+        t0, t1 = i * B, min((i + 1) * B, L)
         go = res["out"][o + t0:o + t1, h].float().cpu().numpy().astype(np.float64)
         gl = res["lse"][h, o + t0:o + t1].cpu().numpy().astype(np.float64)
         e_o = out_error(go, ro[t0:t1, 0])
@@ -222,7 +223,7 @@ def _check_workload(w, samples, every_row=False):
 def _samples(w, heads, per_seq_blocks):
     out = []
     for s, L in enumerate(w.seqlens):
-        nb = math.ceil(L / 128)
+        nb = math.ceil(L / w.block_size)
         blocks = sorted({min(nb - 1, x) for x in per_seq_blocks(nb)})
         for h in heads:
             for i in blocks:
@@ -233,6 +234,14 @@ def _samples(w, heads, per_seq_blocks):
 def test_fullsize_qwen32k():
     w = I.workload("qwen32k")
     _check_workload(w, _samples(w, (0, 13, 31), lambda nb: (0, 1, 5, nb // 2, nb - 2, nb - 1)), every_row=True)
+
+
+def test_fullsize_qwen32k_64_token_blocks():
+    """The 32K workload with 64-token blocks (512 blocks per row): every list
+    against the oracle; sampled rows of both halves of attention tiles."""
+    w = I.workload("qwen32k", block_size=64)
+    _check_workload(w, _samples(w, (0, 13, 31), lambda nb: (0, 1, 2, 7, nb // 2, nb // 2 + 1, nb - 2, nb - 1)),
+                    every_row=True)
 
 
 def test_fullsize_long128k_bench_workload():
@@ -250,6 +259,13 @@ def test_fullsize_fp8_varlen_layers(layer):
 def test_fullsize_sweep64k_extremes(rho):
     w = I.workload("sweep64k", keep_ratio=rho)
     _check_workload(w, _samples(w, (7,), lambda nb: (2, nb - 1)), every_row=(rho == 0.1))
+
+
+def test_fullsize_long128k_64_token_blocks():
+    """The bench workload with 64-token blocks (2048 blocks per row), sampled
+    rows."""
+    w = I.workload("long128k", block_size=64)
+    _check_workload(w, _samples(w, (0, 31), lambda nb: (0, 5, nb // 2 + 1, nb - 1)))
 
 
 def test_fullsize_long128k_shared_lists():
