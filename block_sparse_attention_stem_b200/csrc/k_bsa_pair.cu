@@ -337,7 +337,9 @@ __global__ void __launch_bounds__(kPairThreads, 1)
 #pragma unroll
         for (int ch = 0; ch < 2; ++ch) {
           uint32_t w[16];
-          if (diag) {
+          if constexpr (kPolyMask == 0u) {
+            exp_chunk<0u, kFp8>(rr[ch], c2, nm2, ps0, ps1, w);  // one copy of the code for every half
+          } else if (diag) {
             exp_chunk<0u, kFp8>(rr[ch], c2, nm2, ps0, ps1, w);  // masked keys need an exact 0
           } else {
             exp_chunk<kPolyMask, kFp8>(rr[ch], c2, nm2, ps0, ps1, w);
