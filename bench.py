@@ -64,8 +64,10 @@ def parse_args(argv=None):
                          "once: one untimed step of --workload (the command profilers wrap)")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
     ap.add_argument("--separate-select", action="store_true",
-                    help="mode once: stem_score then stem_select (the selection kernel of its own) instead of the "
-                         "fused stem_score_select")
+                    help="mode once: stem_score then stem_select as two calls (stem_score_select runs the same "
+                         "two kernels unless --fused-select)")
+    ap.add_argument("--fused-select", action="store_true",
+                    help="mode once: stem_score_select with select_mode 1 (the scoring kernel selects its rows)")
     return ap.parse_args(argv)
 
 
@@ -370,8 +372,8 @@ def run_ours(args):
     stream = torch.cuda.current_stream()
 
     def step(ev):
-        # scoring with the selection fused into it (stem_score_select), then
-        # the attention; ev[1] = ev[2] marks the boundary
+        # scoring and selection (stem_score_select: the scoring kernel, then
+        # the selection kernel), then the attention; ev[1] = ev[2] marks the boundary
         ev[0].record(stream)
         b.stem_score_select(qkv, params, scores, vbonus, budgets, row_ptr, col_idx, ws, stream)
         ev[1].record(stream)
@@ -557,9 +559,10 @@ def run_ours(args):
                           f"(first {rows[:3]}...): fp64 block-score row, budget, top-k, attention row; "
                           f"{sec:.1f} s, {fl / 1e9:.1f} GFLOP")}
 
-    # per launch batch of up to 8 sequences: v-norm, budgets, scoring (which
-    # selects) and attention; a separate selection pass when it cannot fuse
-    fused = w.list_mode == 0 and pl.nb_max <= 5888
+    # per launch batch of up to 8 sequences: v-norm, budgets, scoring, the
+    # selection pass and attention (the selection runs in the scoring kernel
+    # only with select_mode 1, which the step does not use)
+    fused = params.select_mode == 1 and w.list_mode == 0 and pl.nb_max <= 5888
     # (fp8: plus one V widening pass per attention call)
     launches_per_step = ((4 if fused else 5) * math.ceil(len([L for L in w.seqlens if L > 0]) / 8)
                          + (1 if w.dtype == "fp8" else 0))
@@ -894,7 +897,7 @@ def run_once(args):
     inp = I.make_inputs(w, device="cuda")
     qkv = b.make_qkv(inp["q"], inp["k"], inp["v"], w.cu_seqlens(), q_scale=inp["q_scale"], k_scale=inp["k_scale"],
                      v_scale=inp["v_scale"], cu_seqlens_dev=inp["cu_seqlens"])
-    params = b.make_params(**w.params())
+    params = b.make_params(**w.params(), select_mode=1 if args.fused_select else 0)
     if args.separate_select:
         scores, _, ws = b.stem_score(qkv, params)
         budgets, row_ptr, col_idx, _ = b.stem_select(qkv, params, scores, ws=ws)

@@ -37,7 +37,7 @@ class StemParams(ctypes.Structure):
                 ("norm", ctypes.c_double), ("beta", ctypes.c_double), ("keep_ratio", ctypes.c_double),
                 ("mu", ctypes.c_double), ("sink_blocks", ctypes.c_int32), ("window_blocks", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_double), ("budget_mode", ctypes.c_int32), ("bonus_mode", ctypes.c_int32),
-                ("list_mode", ctypes.c_int32)]
+                ("list_mode", ctypes.c_int32), ("select_mode", ctypes.c_int32)]
 
 
 class StemQKV(ctypes.Structure):
@@ -110,9 +110,10 @@ def _check(code: int, where: str):
 
 def make_params(block_size=128, stride=8, chunk_size=2048, norm=1.0, beta=0.2, keep_ratio=0.25, mu=0.7,
                 sink_blocks=4, window_blocks=4, softmax_scale=0.0, budget_mode=0, bonus_mode=0,
-                list_mode=0) -> StemParams:
+                list_mode=0, select_mode=0) -> StemParams:
     return StemParams(block_size, stride, chunk_size, float(norm), float(beta), float(keep_ratio), float(mu),
-                      sink_blocks, window_blocks, float(softmax_scale), budget_mode, bonus_mode, list_mode)
+                      sink_blocks, window_blocks, float(softmax_scale), budget_mode, bonus_mode, list_mode,
+                      select_mode)
 
 
 def _ptr(t):
@@ -210,7 +211,7 @@ def stem_select(qkv: QKV, params: StemParams, scores, budgets=None, row_ptr=None
 
 def stem_score_select(qkv: QKV, params: StemParams, scores=None, vbonus=None, budgets=None, row_ptr=None,
                       col_idx=None, ws=None, stream=None):
-    """stem_score then stem_select in one pass (the scoring CTAs select their rows)."""
+    """stem_score then stem_select in one call (in one pass when params.select_mode is 1)."""
     pl = stem_plan(qkv, params)
     dev = qkv.q.device
     hq, hkv = qkv.q.shape[1], qkv.k.shape[1]

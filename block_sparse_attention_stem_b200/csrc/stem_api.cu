@@ -75,6 +75,7 @@ stem_status_t validate(const stem_qkv_t* qkv, const stem_params_t* p) {
   if (p->budget_mode != STEM_BUDGET_RELATIVE && p->budget_mode != STEM_BUDGET_ABSOLUTE) return STEM_ERR_INVALID_ARG;
   if (p->bonus_mode != STEM_BONUS_LOG && p->bonus_mode != STEM_BONUS_STANDARDIZED) return STEM_ERR_INVALID_ARG;
   if (p->list_mode != STEM_LIST_PER_HEAD && p->list_mode != STEM_LIST_PER_GROUP) return STEM_ERR_INVALID_ARG;
+  if (p->select_mode != STEM_SELECT_SEPARATE && p->select_mode != STEM_SELECT_FUSED) return STEM_ERR_INVALID_ARG;
   return STEM_OK;
 }
 
@@ -313,9 +314,12 @@ stem_status_t run_score(const stem_qkv_t* qkv, const stem_params_t* p, const Pla
 }
 
 // The scoring kernel selects the rows it scored (no separate selection pass)
-// for per-head lists whose rows fit its scratch.
+// when asked to, for per-head lists whose rows fit its scratch.  Separate is
+// the default: one warp per list over every list at once finishes sooner
+// than each scoring CTA selecting its own rows after its last key tile.
 bool fuse_selection(const stem_params_t* p, const Plan& pl) {
-  return p->list_mode == STEM_LIST_PER_HEAD && pl.pub.nb_max <= kFusedSelectMaxBlocks;
+  return p->select_mode == STEM_SELECT_FUSED && p->list_mode == STEM_LIST_PER_HEAD &&
+         pl.pub.nb_max <= kFusedSelectMaxBlocks;
 }
 
 stem_status_t run_select(const stem_qkv_t* qkv, const stem_params_t* p, const Plan& pl, int hk0, int nhk,

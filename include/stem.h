@@ -92,6 +92,13 @@ typedef enum {
                               -inf) and written to every query head of the group */
 } stem_list_mode_t;
 
+/* Where the top-k selection runs (the results are the same, bit for bit). */
+typedef enum {
+  STEM_SELECT_SEPARATE = 0,  /* a selection kernel, one warp per list, after the scoring kernel */
+  STEM_SELECT_FUSED = 1      /* the scoring CTAs select the rows they scored, after their last key
+                                tile (per-head lists of at most 5888 blocks; otherwise as SEPARATE) */
+} stem_select_mode_t;
+
 /* Method parameters (AngelSlim documentation §6 defaults in brackets). */
 typedef struct {
   int32_t block_size;     /* block of the scores, lists and attention [128]: 128 or 64 (the
@@ -110,6 +117,7 @@ typedef struct {
   int32_t budget_mode;    /* stem_budget_mode_t */
   int32_t bonus_mode;     /* stem_bonus_mode_t [STEM_BONUS_LOG] */
   int32_t list_mode;      /* stem_list_mode_t [STEM_LIST_PER_HEAD] */
+  int32_t select_mode;    /* stem_select_mode_t [STEM_SELECT_SEPARATE]; no effect on results */
 } stem_params_t;
 
 /* Query/key/value description shared by all calls. */
@@ -206,11 +214,12 @@ STEM_API stem_status_t stem_select(const stem_qkv_t* qkv, const stem_params_t* p
                           const float* scores, int32_t* budgets, int32_t* row_ptr,
                           int32_t* col_idx, void* ws, size_t ws_bytes, stem_stream_t stream);
 
-/* stem_score and stem_select in one pass: same arguments and outputs as the two
+/* stem_score and stem_select in one call: same arguments and outputs as the two
  * calls (scores, vbonus, budgets, row_ptr, col_idx), results bit for bit equal.
- * With per-head lists and nb_max <= 5888 each scoring CTA selects the rows it has
- * just scored (the budgets run first), so the scores are read back from L2 and
- * no separate selection pass runs; otherwise the two passes run in turn. */
+ * With select_mode = STEM_SELECT_FUSED, per-head lists and nb_max <= 5888 each
+ * scoring CTA selects the rows it has just scored (the budgets run first), so
+ * the scores are read back from L2 and no separate selection pass runs;
+ * otherwise (the default) the two passes run in turn. */
 STEM_API stem_status_t stem_score_select(const stem_qkv_t* qkv, const stem_params_t* params,
                                 float* scores, float* vbonus,
                                 int32_t* budgets, int32_t* row_ptr, int32_t* col_idx,
@@ -255,7 +264,7 @@ STEM_API stem_status_t stem_bsa_fwd_paged(const stem_qkv_t* qkv, const stem_page
                                  void* ws, size_t ws_bytes, stem_stream_t stream);
 
 /* score -> select -> attention on one stream with no host round trip (the
- * selection fused into the scoring pass as in stem_score_select).
+ * selection placed as in stem_score_select).
  * row_ptr_out / col_idx_out may be NULL (the workspace then holds the lists);
  * ws_bytes >= plan.ws_prefill_bytes. */
 STEM_API stem_status_t stem_prefill(const stem_qkv_t* qkv, const stem_params_t* params,

@@ -139,6 +139,8 @@ def test_validation_rejects_bad_parameters():
     b.stem_plan(qkv, P(bonus_mode=1))  # the standardized bonus is valid
     assert _status(lambda: b.stem_plan(qkv, P(list_mode=2))) == 1
     b.stem_plan(qkv, P(list_mode=1))  # GQA-shared lists are valid
+    b.stem_plan(qkv, P(select_mode=1))  # the selection inside the scoring kernel is valid
+    assert _status(lambda: b.stem_plan(qkv, P(select_mode=2))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(stride=3))) == 1
     assert _status(lambda: b.stem_plan(qkv, P(stride=16))) == 2
     b.stem_plan(qkv, P(block_size=64))  # 64-token blocks are valid

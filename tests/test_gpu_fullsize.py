@@ -34,8 +34,9 @@ if not torch.cuda.is_available():
 
 
 def _run(w):
-    """The bench's step (stem_score_select, then stem_bsa_fwd); the separate
-    passes (stem_score, then stem_select) must give the same scores and lists."""
+    """The bench's step (stem_score_select, then stem_bsa_fwd); the selection
+    inside the scoring kernel (select_mode 1) must give the same scores and
+    lists."""
     inp = I.make_inputs(w, device="cuda")
     qkv = make_gpu_qkv(b, inp, w.cu_seqlens())
     params = b.make_params(**w.params())
@@ -43,8 +44,7 @@ def _run(w):
     out, lse, _ = b.stem_bsa_fwd(qkv, params, row_ptr, col_idx, ws=ws)
     torch.cuda.synchronize()
     assert b.stem_read_device_status(ws) == 0
-    s2, _, ws2 = b.stem_score(qkv, params)
-    _, rp2, ci2, _ = b.stem_select(qkv, params, s2, ws=ws2)
+    s2, _, rp2, ci2, ws2 = b.stem_score_select(qkv, b.make_params(**w.params(), select_mode=1))
     torch.cuda.synchronize()
     assert b.stem_read_device_status(ws2) == 0
     assert torch.equal(s2.view(torch.int32), scores.view(torch.int32))

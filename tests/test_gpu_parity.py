@@ -116,13 +116,16 @@ def test_select_is_bit_exact_on_identical_fp32_scores(name):
 
 
 @pytest.mark.parametrize("name", list(CASES))
-def test_score_select_equals_score_then_select(name):
-    """The fused pass (scoring CTAs selecting their own rows) gives exactly the
-    two separate passes' scores and lists."""
+@pytest.mark.parametrize("select_mode", [0, 1])
+def test_score_select_equals_score_then_select(name, select_mode):
+    """stem_score_select gives exactly the two separate calls' scores and
+    lists, with the selection kernel after the scoring kernel (select_mode 0)
+    and with the scoring CTAs selecting their own rows (select_mode 1)."""
     c = get_case(name)
     scores, vbonus, ws = b.stem_score(c.qkv, c.params)
     gb, grp, gci, _ = b.stem_select(c.qkv, c.params, scores)
-    s2, gb2, grp2, gci2, ws2 = b.stem_score_select(c.qkv, c.params)
+    params = b.make_params(**c.w.params(), select_mode=select_mode)
+    s2, gb2, grp2, gci2, ws2 = b.stem_score_select(c.qkv, params)
     torch.cuda.synchronize()
     assert b.stem_read_device_status(ws2) == 0
     assert torch.equal(s2.view(torch.int32), scores.view(torch.int32))
