@@ -47,6 +47,15 @@
 // Half h uses K slot and V slot h % 2: K_{h+2} may overwrite K_h once S_h is
 // complete, V_{h+2} may overwrite V_h once P_h V_h is, so a product needs one
 // commit.  Block lists are staged in shared memory; every wait is bounded.
+//
+// 64-token blocks (the "64x128" KV blocks of the HPC-BSA article §3.1): a
+// tcgen05.mma with M = 64 takes as long as one with M = 128, so the CTA keeps
+// its 128-row tile and gives it query blocks 2p and 2p + 1 (rows 0-63 and
+// 64-127).  Their two lists are staged as bitmaps of key blocks, and the CTA
+// walks the union in ascending order, one 64-key unit per listed block, with
+// the same S / P / P V pipeline as the halves above.  A unit in only one of
+// the lists is a block of -inf scores for the other block's rows: those warps
+// store P = 0 and skip the exponentials.
 #include "stem_bsa_common.cuh"
 
 namespace stem {
