@@ -31,6 +31,7 @@ CASES = {
     "mha": W([700], 2, 2, seed=38),  # one query head per KV head
     "std_bonus": W([1000, 128, 2088], 8, 2, seed=36, bonus_mode=1),  # per-KV-head z-score per group
     "group_lists": W([1000, 2088], 8, 2, seed=37, list_mode=1),  # the separate selection pass
+    "b64_varlen": W([1000, 128, 2088, 63], 8, 2, seed=39, block_size=64),  # 64-token blocks
 }
 
 
