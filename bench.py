@@ -63,6 +63,8 @@ def parse_args(argv=None):
                          "variants: the 128K step with the standardized bonus, KV-group-shared lists and 64-token blocks; "
                          "once: one untimed step of --workload (the command profilers wrap)")
     ap.add_argument("--layers", type=int, default=36, help="layers of the fp8 stack")
+    ap.add_argument("--block-size", type=int, choices=[64, 128], default=None,
+                    help="block size of the workload (default: the workload's, 128)")
     ap.add_argument("--separate-select", action="store_true",
                     help="mode once: stem_score then stem_select as two calls (stem_score_select runs the same "
                          "two kernels unless --fused-select)")
@@ -255,8 +257,14 @@ def measure_gemm_peaks(torch, n: int = 8192, reps: int = 10) -> dict:
 
 
 def bench_workload(I, args):
-    """The named workload, with its arithmetic type overridden by --dtype."""
-    return I.workload(args.workload, **({"dtype": args.dtype} if args.dtype else {}))
+    """The named workload, with its arithmetic type overridden by --dtype and
+    its block size by --block-size."""
+    over = {}
+    if args.dtype:
+        over["dtype"] = args.dtype
+    if getattr(args, "block_size", None):
+        over["block_size"] = args.block_size
+    return I.workload(args.workload, **over)
 
 
 def describe(w) -> dict:
@@ -458,7 +466,7 @@ def run_ours(args):
     # attention kernel timed alone, against the fp8 peak (2 x bf16, nominal)
     fp8_attn = None
     if w.dtype == "bf16" and not args.no_fp8:
-        w8 = I.workload(w.name, dtype="fp8")
+        w8 = I.workload(w.name, dtype="fp8", block_size=w.block_size)
         inp8 = I.make_inputs(w8, seed=seed, device="cuda")
         qkv8 = b.make_qkv(inp8["q"], inp8["k"], inp8["v"], w8.cu_seqlens(), q_scale=inp8["q_scale"],
                           k_scale=inp8["k_scale"], v_scale=inp8["v_scale"], cu_seqlens_dev=inp8["cu_seqlens"])
@@ -532,6 +540,8 @@ def run_ours(args):
 
     achieved = pl.attn_flops / (bsa_ms * 1e-3) / 1e12
     traffic_key = w.name if w.dtype == I.workload(w.name).dtype else f"{w.name}:{w.dtype}"
+    if w.block_size != I.workload(w.name).block_size:
+        traffic_key += f":b{w.block_size}"
     traffic = bsa_traffic_per_launch(traffic_key)
     if w.dtype == "fp8":
         roofline = {"bound": "tensor", "kernel": "bsa_kernel", "achieved": round(achieved, 2), "peak": peak_fp8,
