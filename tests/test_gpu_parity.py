@@ -259,6 +259,28 @@ def test_malformed_list_entries_are_skipped_and_reported_64_token_blocks():
     check_attention(out, lse, ro, rl, "bf16")
 
 
+def test_64_token_tiles_with_disjoint_lists():
+    """Every unit of every tile belongs to one of its two query blocks only:
+    block 2p lists its even blocks, block 2p + 1 its odd blocks (both end at
+    their diagonal), so each unit is a -inf block for half of the tile's
+    rows."""
+    c = get_case("b64_varlen")
+    seqs, nbtot = O.seq_blocks(c.cu, 64)
+    rows = []
+    for h in range(c.w.num_q_heads):
+        for (_, _, nb, g0) in seqs:
+            for i in range(nb):
+                rows.append(list(range(i % 2, i + 1, 2)))
+    rp = np.zeros(len(rows) + 1, dtype=np.int64)
+    rp[1:] = np.cumsum([len(r) for r in rows])
+    ci = np.array([j for r in rows for j in r], dtype=np.int64)
+    out, lse, ws = b.stem_bsa_fwd(c.qkv, c.params, torch.from_numpy(rp.astype(np.int32)).cuda(),
+                                  torch.from_numpy(ci.astype(np.int32)).cuda())
+    assert b.stem_read_device_status(ws) == 0
+    ro, rl = O.bsa(c.q, c.k, c.v, c.cu, rp, ci, c.p)
+    check_attention(out, lse, ro, rl, c.w.dtype)
+
+
 @pytest.mark.parametrize("name", ["tiny", "b64_varlen"])
 def test_empty_rows_give_zero_output_and_minus_inf_lse(name):
     c = get_case(name)
