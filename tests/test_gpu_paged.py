@@ -56,6 +56,7 @@ CASES = {
     # 64-token blocks: every 64-key unit is one page lookup
     "b64_page64": (W([1000, 128, 2088, 63], 8, 2, seed=54, block_size=64), 64),
     "b64_fp8_page128": (W([640, 2112, 77], 4, 2, dtype="fp8", seed=55, block_size=64), 128),
+    "b64_shared_lists_page64": (W([1000, 2088], 8, 2, seed=56, block_size=64, list_mode=1), 64),
 }
 
 

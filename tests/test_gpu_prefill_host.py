@@ -35,12 +35,13 @@ CASES = {
 }
 
 
-@pytest.mark.parametrize("name", list(CASES))
-def test_prefill_host_matches_prefill(name):
+@pytest.mark.parametrize("name,select_mode", [(n, 0) for n in CASES] + [("varlen_gqa4", 1), ("fp8_varlen", 1)])
+def test_prefill_host_matches_prefill(name, select_mode):
+    """select_mode 1: each KV-head group's scoring kernel also selects its rows."""
     w = CASES[name]
     inp = I.make_inputs(w, device="cuda")
     qkv = make_gpu_qkv(b, inp, w.cu_seqlens())
-    params = b.make_params(**w.params())
+    params = b.make_params(**w.params(), select_mode=select_mode)
     out_ref, lse_ref, _, _, _ = b.stem_prefill(qkv, params, return_lists=False)
     torch.cuda.synchronize()
     # host copies of the inputs; the device input tensors are overwritten by the call

@@ -22,18 +22,19 @@ if not torch.cuda.is_available():
     pytest.skip("no CUDA device", allow_module_level=True)
 
 
-def _case(seed, dtype="bf16", block_size=128):
+def _case(seed, dtype="bf16", block_size=128, select_mode=0):
     w = I.Workload(name="noalloc", seqlens=[3000, 1000, 640], num_q_heads=8, num_kv_heads=2, dtype=dtype,
                    seed=seed, keep_ratio=0.3, mu=0.7, beta=0.2, sink_blocks=1, window_blocks=2,
                    block_size=block_size)
     dinp = to_device(I.make_inputs(w))
-    return w, make_gpu_qkv(b, dinp, w.cu_seqlens()), b.make_params(**w.params())
+    return w, make_gpu_qkv(b, dinp, w.cu_seqlens()), b.make_params(**w.params(), select_mode=select_mode)
 
 
-@pytest.mark.parametrize("dtype,block_size", [("bf16", 128), ("fp8", 128), ("bf16", 64)])
-def test_noalloc_matches_workspace_prefill_on_two_calls(dtype, block_size):
+@pytest.mark.parametrize("dtype,block_size,select_mode", [("bf16", 128, 0), ("fp8", 128, 0), ("bf16", 64, 0),
+                                                          ("bf16", 128, 1)])
+def test_noalloc_matches_workspace_prefill_on_two_calls(dtype, block_size, select_mode):
     for seed in (101, 202):
-        w, qkv, params = _case(seed, dtype, block_size)
+        w, qkv, params = _case(seed, dtype, block_size, select_mode)
         ref_out, ref_lse, ref_rp, ref_ci, ws = b.stem_prefill(qkv, params)
         out, lse, rp, ci = b.stem_prefill_noalloc(qkv, params)
         torch.cuda.synchronize()
